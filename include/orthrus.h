@@ -1,0 +1,228 @@
+/*
+ * orthrus.h - C ABI of the B200 (sm_100a) Orthrus dual-view decode step.
+ *
+ * Orthrus ("Memory-Efficient Parallel Token Generation via Dual-View
+ * Diffusion"; opentrain.ai abstract, atlas.scime.ai summary "Approach")
+ * augments a frozen autoregressive (AR) decoder with a trainable attention
+ * path per layer. One decode step:
+ *   1. draft view: one forward over the block [y, MASK x (K-1)] with the draft
+ *      attention module; every block position attends to the frozen model's
+ *      KV cache and to all block positions (bidirectional); the argmax of block
+ *      row i is the draft d_{i+1}                      -> orthrus_draft_block
+ *   2. verify view: one causal forward of the frozen model over [y, d_1..d_K];
+ *      the argmax of block row j is g_j; the block's base K/V is written into
+ *      cache slots n..n+K                               -> orthrus_verify_block
+ *   3. greedy consensus: a = number of leading d_i == g_{i-1}; commit
+ *      d_1..d_a and g_a; slots n..n+a become live; n += a+1; y = g_a
+ *                                                       -> orthrus_accept_commit
+ * (Hacker News summary "Idea": the diffusion head projects K tokens in
+ * parallel and the AR head verifies in a second pass, accepting the longest
+ * matching prefix; news article "KV Cache Overhead": one shared cache, only
+ * the AR view updates it.) orthrus_decode_step runs all three.
+ *
+ * Conventions used by every call:
+ *   - All device memory is owned and allocated by the caller. The library
+ *     allocates nothing: the per-model "plan" is a caller-provided HOST buffer
+ *     of orthrus_plan_bytes() bytes, and all scratch lives in a caller-provided
+ *     DEVICE workspace of orthrus_workspace_bytes() bytes.
+ *   - Every call is asynchronous on the given CUDA stream and performs no host
+ *     synchronisation; results are valid once the stream reaches them.
+ *   - Host-detectable misuse (NULL pointers, sizes out of range) returns an
+ *     error before anything is launched. Conditions found on the device
+ *     (cache overrun, NaN logits, a bounded wait that ran out) are recorded in
+ *     a sticky device int32 status word (first error wins), readable through
+ *     orthrus_status_ptr(); kernels then stop writing the cache.
+ *   - Matrices are row-major. bf16 = IEEE bfloat16 bits (uint16).
+ *   - Model layout: W_qkv rows = q heads | k heads | v heads (each head_dim rows);
+ *     W_gate_up rows = gate (d_ff) | up (d_ff); W_o [d_model][n_heads*head_dim];
+ *     W_down [d_model][d_ff]; embed and lm_head [vocab][d_model] (untied).
+ *   - KV cache: K and V bf16 [n_layers][batch][n_kv_heads][capacity][head_dim],
+ *     post-QK-norm and post-RoPE; cache.len[b] (device int32) = live slots.
+ *   - Shapes supported by the kernels: head_dim in {64, 128}; d_model, d_ff and
+ *     n_heads*head_dim multiples of 128; vocab a multiple of 128;
+ *     n_heads / n_kv_heads in {1, 2, 4, 8}; 1 <= K <= 64.
+ */
+#ifndef ORTHRUS_H
+#define ORTHRUS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* orthrus_stream; /* same type as cudaStream_t */
+
+typedef enum {
+  ORTHRUS_OK = 0,
+  ORTHRUS_ERR_ARG = 1,         /* NULL pointer, size or shape out of range                */
+  ORTHRUS_ERR_CAPACITY = 2,    /* len + block > cache capacity (host or device detected)  */
+  ORTHRUS_ERR_CUDA = 3,        /* a CUDA runtime call failed                               */
+  ORTHRUS_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out (device status only) */
+  ORTHRUS_ERR_NAN = 5,         /* a NaN logit reached an argmax (device status only)      */
+  ORTHRUS_ERR_UNSUPPORTED = 6, /* shape outside what the kernels implement                */
+  ORTHRUS_ERR_WORKSPACE = 7    /* plan or workspace buffer too small                       */
+} orthrus_status;
+
+/* Decoder shape (Qwen3-style: pre-RMSNorm, optional per-head q/k RMSNorm,
+ * rotate-half RoPE at absolute positions, SwiGLU MLP). mask_id is the token
+ * placed at draft-block positions 2..K. */
+typedef struct {
+  int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, d_ff, vocab, mask_id, qk_norm;
+  float rope_theta, rms_eps;
+} orthrus_config;
+
+/* Device pointers to the weights. Per-layer members are HOST arrays of
+ * n_layers DEVICE pointers. Norm gains are fp32; matrices are bf16.
+ * wd_* are the draft attention module's own projections and q/k norm gains;
+ * the draft view reuses attn_norm, mlp_norm, the MLP, final_norm and lm_head. */
+typedef struct {
+  const void* embed;      /* bf16 [vocab][d_model]     */
+  const float* final_norm; /* fp32 [d_model]            */
+  const void* lm_head;    /* bf16 [vocab][d_model]     */
+  const float* const* attn_norm; /* [L] fp32 [d_model]  */
+  const float* const* mlp_norm;  /* [L] fp32 [d_model]  */
+  const void* const* w_qkv;      /* [L] bf16 [(H+2Hkv)d][d_model] */
+  const void* const* w_o;        /* [L] bf16 [d_model][H d]       */
+  const float* const* q_norm;    /* [L] fp32 [d] (unused if !qk_norm) */
+  const float* const* k_norm;    /* [L] fp32 [d]                  */
+  const void* const* w_gate_up;  /* [L] bf16 [2 d_ff][d_model]    */
+  const void* const* w_down;     /* [L] bf16 [d_model][d_ff]      */
+  const void* const* wd_qkv;     /* [L] bf16, shape of w_qkv      */
+  const void* const* wd_o;       /* [L] bf16, shape of w_o        */
+  const float* const* wd_q_norm; /* [L] fp32 [d]                  */
+  const float* const* wd_k_norm; /* [L] fp32 [d]                  */
+} orthrus_weights;
+
+/* The one shared KV cache (base view only). */
+typedef struct {
+  void* k;        /* bf16 [L][batch][Hkv][capacity][d] */
+  void* v;        /* bf16 [L][batch][Hkv][capacity][d] */
+  int32_t* len;   /* device int32 [batch]: live slots per sequence */
+  int32_t batch;
+  int32_t capacity;
+} orthrus_cache;
+
+/* ---- set-up ------------------------------------------------------------ */
+
+/* Host bytes the plan needs (TMA descriptors for every weight, the cache and
+ * the workspace, plus launch geometry). */
+size_t orthrus_plan_bytes(const orthrus_config* cfg);
+
+/* Device bytes of the workspace for a plan with this batch, cache capacity,
+ * block size limit max_block (1 <= K <= max_block <= 64) and row limit
+ * max_rows (rows of one forward: at least batch*(max_block+1); prefill runs
+ * in causal chunks of at most max_rows tokens). 0 for an invalid request.
+ * Includes the draft view's block scratch, 2 * L * batch * max_block * Hkv *
+ * d * 2 bytes: 4.5 MiB at the Qwen3-8B shape with K = 32 and batch 1, the
+ * pages' "about 4.5 MiB, flat" KV overhead (Hacker News summary "Results"). */
+size_t orthrus_workspace_bytes(const orthrus_config* cfg, int32_t batch, int32_t capacity, int32_t max_block,
+                               int32_t max_rows);
+
+/* Byte offset of the draft block scratch (K part, then V part) inside the
+ * workspace, and its total size (K and V). */
+size_t orthrus_block_scratch_offset(const orthrus_config* cfg, int32_t batch, int32_t capacity, int32_t max_block,
+                                    int32_t max_rows);
+size_t orthrus_block_scratch_bytes(const orthrus_config* cfg, int32_t batch, int32_t max_block);
+
+/* Fill the caller's host buffer `plan` for these weights, cache and workspace
+ * and zero the workspace on `stream`. Pointers are captured: weights, cache
+ * and workspace must stay allocated, at the same addresses, while the plan is
+ * used. Errors: ORTHRUS_ERR_ARG, ORTHRUS_ERR_UNSUPPORTED, ORTHRUS_ERR_WORKSPACE,
+ * ORTHRUS_ERR_CUDA. */
+orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_config* cfg,
+                                 const orthrus_weights* w, const orthrus_cache* cache, int32_t max_block,
+                                 int32_t max_rows, void* workspace, size_t workspace_bytes, orthrus_stream stream);
+
+/* Device pointer to the sticky int32 status word (inside the workspace), and
+ * a call that resets it to ORTHRUS_OK on `stream`. */
+int32_t* orthrus_status_ptr(const void* plan);
+orthrus_status orthrus_clear_status(const void* plan, orthrus_stream stream);
+
+/* Number of kernels one call of orthrus_decode_step launches for block size K
+ * (planted drafts add one device-to-device copy, not a kernel). */
+int32_t orthrus_decode_step_launches(const void* plan, int32_t K);
+
+/* ---- the decode step ---------------------------------------------------- */
+
+/* AR prefill (atlas summary "Approach": the frozen backbone does prefill and
+ * builds the KV cache). tokens: device int32 [batch][max_prompt];
+ * prompt_len: HOST int32 [batch], 1 <= prompt_len[b] <= max_prompt. Writes the
+ * prompt's K/V to slots [0, prompt_len[b]), sets cache.len[b] = prompt_len[b]
+ * and pending[b] (device int32 [batch]) = argmax at the last prompt row: the
+ * first generated token. Runs causal chunks of at most max_rows tokens.
+ * Errors: ORTHRUS_ERR_ARG; ORTHRUS_ERR_CAPACITY if a prompt exceeds capacity. */
+orthrus_status orthrus_prefill(const void* plan, const int32_t* tokens, const int32_t* prompt_len, int32_t max_prompt,
+                               int32_t* pending, orthrus_stream stream);
+
+/* Draft view (atlas summary "Approach": predict a block of K tokens in one
+ * forward over the same KV cache). pending: device int32 [batch]. Writes
+ * draft (device int32 [batch][K]) with d_1..d_K. logits (nullable): device
+ * fp32 [batch][K][vocab] of the draft rows, for checking. The cache is read,
+ * never written; the block's draft-view K/V stays in the block scratch. */
+orthrus_status orthrus_draft_block(const void* plan, const int32_t* pending, int32_t K, int32_t* draft, float* logits,
+                                   orthrus_stream stream);
+
+/* Verify view (HN summary "Idea": the AR head verifies in a second pass).
+ * Causal forward of the frozen model over [pending, draft[0..K-1]] at
+ * positions len..len+K. Writes ar_argmax (device int32 [batch][K+1]) with
+ * g_0..g_K and the block's base K/V into cache slots [len, len+K]; len is not
+ * changed. K = 0 is plain greedy AR decoding of one token. logits (nullable):
+ * fp32 [batch][K+1][vocab]. Device error ORTHRUS_ERR_CAPACITY if
+ * len + K + 1 > capacity (the block is then not written). */
+orthrus_status orthrus_verify_block(const void* plan, const int32_t* pending, const int32_t* draft, int32_t K,
+                                    int32_t* ar_argmax, float* logits, orthrus_stream stream);
+
+/* Greedy consensus and KV commit (HN summary "Idea": accept the longest
+ * matching prefix; opentrain.ai abstract: exact consensus). Per sequence:
+ * a = number of leading i with draft[i-1] == ar_argmax[i-1]; committed[b] =
+ * d_1..d_a, g_a, then -1 up to K+1 entries; accept_len[b] = a;
+ * cache.len[b] += a + 1; pending[b] = g_a. With poison_dead != 0 the dead
+ * verify slots [len+a+1, len+K] of every layer are overwritten with NaN
+ * (a check that nothing reads past len). All device int32 arrays. */
+orthrus_status orthrus_accept_commit(const void* plan, int32_t* pending, const int32_t* draft,
+                                     const int32_t* ar_argmax, int32_t K, int32_t* accept_len, int32_t* committed,
+                                     int32_t poison_dead, orthrus_stream stream);
+
+/* One full Orthrus step: draft view, (planted drafts copied over the draft
+ * view's output when `planted` is not NULL: device int32 [batch][K]), verify
+ * view, accept/commit. pending is updated in place; accept_len [batch] and
+ * committed [batch][K+1] as in orthrus_accept_commit. */
+orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K, const int32_t* planted,
+                                   int32_t* accept_len, int32_t* committed, orthrus_stream stream);
+
+/* ---- single kernels, exposed for parity tests and microbenchmarks ------ */
+
+/* Block attention (the K1 kernel alone) for one layer's cache:
+ *   q        bf16 [batch][Hkv][Q*G][d]: row i*G + g is query head kvh*G+g at block position i
+ *            (post-norm, post-RoPE);
+ *   k_cache, v_cache  bf16 [batch][Hkv][capacity][d];
+ *   k_blk, v_blk      bf16 [batch][Hkv][blk_stride][d] (draft mode only: the
+ *            block's own K/V, blk_stride >= Q);
+ *   len      device int32 [batch]: cache rows [0, len[b]) precede the block;
+ *   mode 0 = draft: every row sees cache[0,len) and block rows [0,Q);
+ *   mode 1 = verify: the block's K/V already sit in cache slots [len, len+Q);
+ *            row i sees cache[0, len+i].
+ *   out      bf16 [batch][Q][H*d] (token-major, head h at columns h*d..).
+ * Scratch comes from `workspace` (orthrus_attention_workspace_bytes). */
+size_t orthrus_attention_workspace_bytes(int32_t batch, int32_t n_kv_heads, int32_t group, int32_t Q, int32_t head_dim,
+                                         int32_t capacity);
+orthrus_status orthrus_attention(const void* q, const void* k_cache, const void* v_cache, const void* k_blk,
+                                 const void* v_blk, const int32_t* len, int32_t batch, int32_t n_kv_heads,
+                                 int32_t group, int32_t Q, int32_t head_dim, int32_t capacity, int32_t blk_stride,
+                                 int32_t mode, void* out, void* workspace, size_t workspace_bytes,
+                                 int32_t* status, orthrus_stream stream);
+
+/* Y[M][N] = X[M][Kd] * W[N][Kd]^T on the tensor cores (the K2 kernel with a
+ * plain fp32 store epilogue). X, W bf16; Y fp32. N a multiple of 128, Kd a
+ * multiple of 64. Scratch from `workspace` (orthrus_linear_workspace_bytes). */
+size_t orthrus_linear_workspace_bytes(int32_t M, int32_t N, int32_t Kd);
+orthrus_status orthrus_linear(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t Kd,
+                              void* workspace, size_t workspace_bytes, int32_t* status, orthrus_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORTHRUS_H */

@@ -1,0 +1,746 @@
+// Host side of liborthrus: plan construction (TMA descriptors encoded once),
+// launch geometry, the forward orchestration of the draft / verify / prefill
+// passes, and the C-ABI entry points declared in include/orthrus.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "attention.cuh"
+#include "gemm.cuh"
+#include "orthrus.h"
+#include "small.cuh"
+
+using namespace orthrus;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// driver entry point for tensor-map encoding (no link against libcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 2D bf16 map over a row-major [rows][cols] matrix; box = box_cols x box_rows, 128-byte swizzle.
+bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f || !base) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 map over [z][rows][cols]; box = 64 cols x 128 rows x 1.
+bool map3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t z) {
+  EncodeTiledFn f = encode_fn();
+  if (!f || !base) return false;
+  cuuint64_t dims[3] = {cols, rows, z};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int round_up(int x, int a) { return (x + a - 1) / a * a; }
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+constexpr size_t kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100
+
+// ---------------------------------------------------------------------------
+// plan
+// ---------------------------------------------------------------------------
+constexpr uint64_t kPlanMagic = 0x4F52544852555331ull;  // "ORTHRUS1"
+enum { M_WQKV = 0, M_WO, M_WGU, M_WDOWN, M_WDQKV, M_WDO, M_PER_LAYER };
+enum { G_LM = 0, G_XN, G_ATTN, G_ACT, G_Q, G_KC, G_VC, G_KB, G_VB, G_COUNT };
+
+struct LayerPtrs {
+  const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
+  const void *w_qkv, *w_o, *w_gu, *w_down, *wd_qkv, *wd_o;
+};
+
+struct alignas(64) Plan {
+  uint64_t magic;
+  orthrus_config cfg;
+  int L, B, cap, max_block, max_rows, sms, chunk_keys, attn_slots;
+  const void* embed;
+  const float* final_norm;
+  const void* lm_head;
+  __nv_bfloat16 *kc, *vc;
+  int* len;
+  void* ws;
+  size_t ws_bytes;
+  int* status;
+  float* h;
+  __nv_bfloat16 *xn, *qbuf, *attn, *act, *blk_k, *blk_v;
+  float2* rope;
+  unsigned long long* amax;
+  int *draft_ids, *ar_ids;
+  float* gemm_part;
+  int* gemm_cnt;
+  float* att_o;
+  float2* att_ml;
+  int* att_cnt;
+  size_t layers_off, maps_off;
+
+  const LayerPtrs& layer(int l) const { return reinterpret_cast<const LayerPtrs*>((const char*)this + layers_off)[l]; }
+  LayerPtrs& layer(int l) { return reinterpret_cast<LayerPtrs*>((char*)this + layers_off)[l]; }
+  const CUtensorMap& lmap(int l, int which) const {
+    return reinterpret_cast<const CUtensorMap*>((const char*)this + maps_off)[l * M_PER_LAYER + which];
+  }
+  CUtensorMap* lmap_mut(int l, int which) {
+    return reinterpret_cast<CUtensorMap*>((char*)this + maps_off) + l * M_PER_LAYER + which;
+  }
+  const CUtensorMap& gmap(int which) const {
+    return reinterpret_cast<const CUtensorMap*>((const char*)this + maps_off)[L * M_PER_LAYER + which];
+  }
+  CUtensorMap* gmap_mut(int which) {
+    return reinterpret_cast<CUtensorMap*>((char*)this + maps_off) + L * M_PER_LAYER + which;
+  }
+};
+
+size_t plan_layout(int L, size_t* layers_off, size_t* maps_off) {
+  size_t off = align_up(sizeof(Plan), 64);
+  *layers_off = off;
+  off = align_up(off + sizeof(LayerPtrs) * (size_t)L, 64);
+  *maps_off = off;
+  off += sizeof(CUtensorMap) * (size_t)(L * M_PER_LAYER + G_COUNT);
+  return off + 64;  // slack for aligning the caller's buffer
+}
+
+Plan* plan_cast(const void* p) {
+  if (!p) return nullptr;
+  Plan* P = (Plan*)(((uintptr_t)p + 63) & ~(uintptr_t)63);
+  return P->magic == kPlanMagic ? P : nullptr;
+}
+
+bool config_ok(const orthrus_config* c) {
+  if (!c) return false;
+  if (c->n_layers < 1 || c->d_model < 128 || c->n_heads < 1 || c->n_kv_heads < 1) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->n_heads % c->n_kv_heads) return false;
+  const int G = c->n_heads / c->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+  if (c->d_model % 128 || c->d_ff % 128 || (c->n_heads * c->head_dim) % 128 || c->vocab % 128) return false;
+  if (((c->n_heads + 2 * c->n_kv_heads) * c->head_dim) % 128) return false;
+  if (c->mask_id < 0 || c->mask_id >= c->vocab) return false;
+  return true;
+}
+
+// Split-KV chunk size for a cache of `cap` keys: chunk boundaries sit at fixed
+// absolute positions for every call made with the same (batch, capacity).
+int attn_chunk_keys(int B, int Hkv, int row_tiles, int cap) {
+  const int sms = num_sms();
+  const int units = std::max(1, B * Hkv * row_tiles);
+  const int target = std::max(1, (2 * sms + units - 1) / units);
+  return round_up(std::max(128, (cap + target - 1) / target), 128);
+}
+
+// workspace layout
+struct WsLayout {
+  size_t status, h, xn, qbuf, attn, act, rope, amax, draft_ids, ar_ids, gemm_part, gemm_cnt, att_o, att_ml, att_cnt,
+      blk_k, blk_v, total;
+  int chunk_keys, attn_slots;
+};
+
+int gemm_counter_count(const orthrus_config* c, int max_rows) {
+  const int mt = (max_rows + 127) / 128;
+  int nt = std::max({c->vocab / 128, c->d_ff / 64, ((c->n_heads + 2 * c->n_kv_heads) * c->head_dim) / 128,
+                     c->d_model / 128});
+  return mt * nt;
+}
+
+WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows, int cap) {
+  WsLayout w{};
+  const int D = c->d_model, Hd = c->n_heads * c->head_dim, F = c->d_ff, d = c->head_dim, L = c->n_layers;
+  const int G = c->n_heads / c->n_kv_heads, Hkv = c->n_kv_heads;
+  const int sms = num_sms();
+  const int rt_dec = (G * (max_block + 1) + 127) / 128;
+  const int ck = attn_chunk_keys(B, Hkv, rt_dec, cap);
+  w.chunk_keys = ck;
+  const int max_chunks = (cap + ck - 1) / ck + 1;
+  const int rt_pre = (G * max_rows + 127) / 128;
+  w.attn_slots = std::max(B * Hkv * rt_dec, Hkv * rt_pre) * max_chunks;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.status = take(256);
+  w.h = take((size_t)max_rows * D * 4);
+  w.xn = take((size_t)max_rows * D * 2);
+  w.qbuf = take((size_t)max_rows * Hd * 2 + 128 * d * 2);
+  w.attn = take((size_t)max_rows * Hd * 2);
+  w.act = take((size_t)max_rows * F * 2);
+  w.rope = take((size_t)max_rows * (d / 2) * 8);
+  w.amax = take((size_t)max_rows * 8);
+  w.draft_ids = take((size_t)B * max_block * 4);
+  w.ar_ids = take((size_t)B * (max_block + 1) * 4);
+  w.gemm_part = take((size_t)2 * sms * 128 * 128 * 4);
+  w.gemm_cnt = take((size_t)gemm_counter_count(c, max_rows) * 4);
+  w.att_o = take((size_t)w.attn_slots * 128 * d * 4);
+  w.att_ml = take((size_t)w.attn_slots * 128 * 8);
+  w.att_cnt = take((size_t)std::max(B * Hkv * rt_dec, Hkv * rt_pre) * 4);
+  const size_t blk = (size_t)L * B * Hkv * max_block * d * 2;
+  w.blk_k = take(blk);
+  w.blk_v = take(blk);
+  w.total = off;
+  return w;
+}
+
+template <typename F>
+bool set_smem_attr(F* kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// launches
+// ---------------------------------------------------------------------------
+template <int EPI>
+cudaError_t launch_gemm(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs a, int N, int Kd, int M,
+                        cudaStream_t st) {
+  a.N = N;
+  a.Kd = Kd;
+  a.M = M;
+  a.m_tiles = (M + 127) / 128;
+  a.Mt = a.m_tiles > 1 ? 128 : round_up(std::max(M, 1), 16);
+  a.mt_alloc = std::max(32, next_pow2(a.Mt));
+  a.n_tiles = (EPI == EPI_SWIGLU) ? N / 128 : N / 128;  // SwiGLU: N = 2F, a tile = 64 gate + 64 up rows
+  a.k_chunks = Kd / 64;
+  a.total_units = (long long)a.m_tiles * a.n_tiles * a.k_chunks;
+  const int G = (int)std::min<long long>(num_sms(), a.total_units);
+  const size_t fixed = gemm_smem_bytes(a.Mt, 0);
+  const size_t stage = 16384 + (size_t)a.Mt * 128;
+  a.stages = (int)std::min<size_t>(12, (kSmemLimit - fixed) / stage);
+  const size_t smem = gemm_smem_bytes(a.Mt, a.stages);
+  static bool attr = false;
+  if (!attr) attr = set_smem_attr(gemm_kernel<EPI>, kSmemLimit);
+  gemm_kernel<EPI><<<G, kGemmThreads, smem, st>>>(tmW, tmX, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tkb, const CUtensorMap& tvb, const AttnArgs& a, cudaStream_t st) {
+  dim3 grid(a.max_chunks, a.row_tiles, a.B * a.Hkv);
+  const size_t smem = attn_smem_bytes(d);
+  if (d == 128) {
+    static bool attr = false;
+    if (!attr) attr = set_smem_attr(attention_kernel<128>, kSmemLimit);
+    attention_kernel<128><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, tkb, tvb, a);
+  } else {
+    static bool attr = false;
+    if (!attr) attr = set_smem_attr(attention_kernel<64>, kSmemLimit);
+    attention_kernel<64><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, tkb, tvb, a);
+  }
+  return cudaGetLastError();
+}
+
+GemmArgs base_gemm_args(const Plan* P) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.partial = P->gemm_part;
+  a.tile_counter = P->gemm_cnt;
+  a.status = P->status;
+  return a;
+}
+
+// One forward over a block of Q rows for sequences [b0, b0+nb).
+//   kind: BLOCK_DRAFT / BLOCK_VERIFY / BLOCK_PREFILL
+//   head: run final norm + LM head + argmax; last_row_only: only row Q-1 of each sequence
+//   argmax_out: [rows of the head] int32; logits: nullable fp32 [rows][vocab]
+orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int* pending, const int* draft,
+                       const int* tokens, int tok_stride, int tok_off, bool head, bool last_row_only, int* argmax_out,
+                       float* logits, cudaStream_t st) {
+  const orthrus_config& c = P->cfg;
+  const int D = c.d_model, H = c.n_heads, Hkv = c.n_kv_heads, d = c.head_dim, F = c.d_ff, V = c.vocab;
+  const int G = H / Hkv, M = nb * Q;
+  const bool draft_view = kind == BLOCK_DRAFT;
+  cudaError_t e;
+
+  EmbedArgs ea;
+  ea.kind = kind;
+  ea.nb = nb;
+  ea.b0 = b0;
+  ea.Q = Q;
+  ea.D = D;
+  ea.d = d;
+  ea.V = V;
+  ea.mask_id = c.mask_id;
+  ea.cap = P->cap;
+  ea.theta = (double)c.rope_theta;
+  ea.pending = pending;
+  ea.draft = draft;
+  ea.tokens = tokens;
+  ea.tok_stride = tok_stride;
+  ea.tok_off = tok_off;
+  ea.len = P->len;
+  ea.embed = (const __nv_bfloat16*)P->embed;
+  ea.h = P->h;
+  ea.rope = P->rope;
+  ea.status = P->status;
+  embed_kernel<<<M, 256, 0, st>>>(ea);
+
+  AttnArgs aa;
+  memset(&aa, 0, sizeof(aa));
+  aa.B = nb;
+  aa.Hkv = Hkv;
+  aa.G = G;
+  aa.Q = Q;
+  aa.d = d;
+  aa.mode = draft_view ? 0 : 1;
+  aa.b0 = b0;
+  aa.rows = Q * G;
+  aa.row_tiles = (aa.rows + 127) / 128;
+  aa.chunk_keys = P->chunk_keys;
+  aa.cap = P->cap;
+  aa.max_chunks = (P->cap + P->chunk_keys - 1) / P->chunk_keys + (draft_view ? 1 : 0);
+  aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+  aa.len = P->len;
+  aa.out = P->attn;
+  aa.part_o = P->att_o;
+  aa.part_ml = P->att_ml;
+  aa.counter = P->att_cnt;
+  aa.status = P->status;
+  if ((long long)nb * Hkv * aa.row_tiles * aa.max_chunks > P->attn_slots) return ORTHRUS_ERR_WORKSPACE;
+
+  for (int l = 0; l < P->L; ++l) {
+    const LayerPtrs& lp = P->layer(l);
+    rmsnorm_kernel<<<M, 256, 0, st>>>(P->h, D, lp.attn_norm, c.rms_eps, P->xn, 0, 1, nullptr);
+
+    GemmArgs g = base_gemm_args(P);
+    g.qkv.H = H;
+    g.qkv.Hkv = Hkv;
+    g.qkv.d = d;
+    g.qkv.Q = Q;
+    g.qkv.b0 = b0;
+    g.qkv.qk_norm = c.qk_norm;
+    g.qkv.mode = draft_view ? VIEW_DRAFT : VIEW_VERIFY;
+    g.qkv.eps = c.rms_eps;
+    g.qkv.gq = draft_view ? lp.wd_q_norm : lp.q_norm;
+    g.qkv.gk = draft_view ? lp.wd_k_norm : lp.k_norm;
+    g.qkv.rope = P->rope;
+    g.qkv.len = P->len;
+    g.qkv.qbuf = P->qbuf;
+    if (draft_view) {
+      const size_t lo = (size_t)l * P->B * Hkv * P->max_block * d;
+      g.qkv.kdst = P->blk_k + lo;
+      g.qkv.vdst = P->blk_v + lo;
+      g.qkv.kv_stride = P->max_block;
+    } else {
+      const size_t lo = (size_t)l * P->B * Hkv * P->cap * d;
+      g.qkv.kdst = P->kc + lo;
+      g.qkv.vdst = P->vc + lo;
+      g.qkv.kv_stride = P->cap;
+    }
+    const int qkv_rows = (H + 2 * Hkv) * d;
+    if ((e = launch_gemm<EPI_QKV>(P->lmap(l, draft_view ? M_WDQKV : M_WQKV), P->gmap(G_XN), g, qkv_rows, D, M, st)) !=
+        cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
+
+    aa.z_cache = l * P->B * Hkv;
+    aa.z_blk = l * P->B * Hkv;
+    if ((e = launch_attention(d, P->gmap(G_Q), P->gmap(G_KC), P->gmap(G_VC), P->gmap(G_KB), P->gmap(G_VB), aa, st)) !=
+        cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
+
+    g = base_gemm_args(P);
+    g.out_f32 = P->h;
+    g.ld_out = D;
+    if ((e = launch_gemm<EPI_RESID>(P->lmap(l, draft_view ? M_WDO : M_WO), P->gmap(G_ATTN), g, D, H * d, M, st)) !=
+        cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
+
+    rmsnorm_kernel<<<M, 256, 0, st>>>(P->h, D, lp.mlp_norm, c.rms_eps, P->xn, 0, 1, nullptr);
+    g = base_gemm_args(P);
+    g.out_bf16 = P->act;
+    g.ld_out = F;
+    g.swiglu_F = F;
+    if ((e = launch_gemm<EPI_SWIGLU>(P->lmap(l, M_WGU), P->gmap(G_XN), g, 2 * F, D, M, st)) != cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
+
+    g = base_gemm_args(P);
+    g.out_f32 = P->h;
+    g.ld_out = D;
+    if ((e = launch_gemm<EPI_RESID>(P->lmap(l, M_WDOWN), P->gmap(G_ACT), g, D, F, M, st)) != cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
+  }
+
+  if (!head) return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
+  const int HR = last_row_only ? nb : M;
+  rmsnorm_kernel<<<HR, 256, 0, st>>>(P->h, D, P->final_norm, c.rms_eps, P->xn, last_row_only ? Q - 1 : 0,
+                                     last_row_only ? Q : 1, P->amax);
+  GemmArgs g = base_gemm_args(P);
+  g.amax = P->amax;
+  g.logits = logits;
+  g.ld_logits = V;
+  if ((e = launch_gemm<EPI_ARGMAX>(P->gmap(G_LM), P->gmap(G_XN), g, V, D, HR, st)) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  argmax_finalize_kernel<<<(HR + 127) / 128, 128, 0, st>>>(P->amax, HR, argmax_out, P->status);
+  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+size_t orthrus_plan_bytes(const orthrus_config* cfg) {
+  if (!config_ok(cfg)) return 0;
+  size_t a, b;
+  return plan_layout(cfg->n_layers, &a, &b);
+}
+
+static bool sizes_ok(const orthrus_config* cfg, int batch, int capacity, int max_block, int max_rows) {
+  return config_ok(cfg) && batch >= 1 && capacity >= 1 && max_block >= 1 && max_block <= 64 &&
+         (long long)max_rows >= (long long)batch * (max_block + 1) && max_rows <= (1 << 20);
+}
+
+size_t orthrus_workspace_bytes(const orthrus_config* cfg, int32_t batch, int32_t capacity, int32_t max_block,
+                               int32_t max_rows) {
+  if (!sizes_ok(cfg, batch, capacity, max_block, max_rows)) return 0;
+  return ws_layout(cfg, batch, max_block, max_rows, capacity).total;
+}
+
+size_t orthrus_block_scratch_offset(const orthrus_config* cfg, int32_t batch, int32_t capacity, int32_t max_block,
+                                    int32_t max_rows) {
+  if (!sizes_ok(cfg, batch, capacity, max_block, max_rows)) return 0;
+  return ws_layout(cfg, batch, max_block, max_rows, capacity).blk_k;
+}
+
+size_t orthrus_block_scratch_bytes(const orthrus_config* cfg, int32_t batch, int32_t max_block) {
+  if (!config_ok(cfg) || batch < 1 || max_block < 1) return 0;
+  return 2ull * cfg->n_layers * batch * max_block * cfg->n_kv_heads * cfg->head_dim * 2ull;
+}
+
+orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_config* cfg, const orthrus_weights* w,
+                                 const orthrus_cache* cache, int32_t max_block, int32_t max_rows, void* workspace,
+                                 size_t workspace_bytes, orthrus_stream stream) {
+  if (!plan || !cfg || !w || !cache || !workspace) return ORTHRUS_ERR_ARG;
+  if (!config_ok(cfg)) return ORTHRUS_ERR_UNSUPPORTED;
+  if (!cache->k || !cache->v || !cache->len) return ORTHRUS_ERR_ARG;
+  if (!sizes_ok(cfg, cache->batch, cache->capacity, max_block, max_rows)) return ORTHRUS_ERR_ARG;
+  const int L = cfg->n_layers;
+  size_t layers_off, maps_off;
+  if (plan_bytes < plan_layout(L, &layers_off, &maps_off)) return ORTHRUS_ERR_WORKSPACE;
+  const WsLayout wl = ws_layout(cfg, cache->batch, max_block, max_rows, cache->capacity);
+  if (workspace_bytes < wl.total) return ORTHRUS_ERR_WORKSPACE;
+  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->mlp_norm || !w->w_qkv || !w->w_o ||
+      !w->w_gate_up || !w->w_down || !w->wd_qkv || !w->wd_o)
+    return ORTHRUS_ERR_ARG;
+  if (cfg->qk_norm && (!w->q_norm || !w->k_norm || !w->wd_q_norm || !w->wd_k_norm)) return ORTHRUS_ERR_ARG;
+  if (!encode_fn()) return ORTHRUS_ERR_CUDA;
+
+  Plan* P = (Plan*)(((uintptr_t)plan + 63) & ~(uintptr_t)63);
+  memset(P, 0, sizeof(Plan));
+  P->cfg = *cfg;
+  P->L = L;
+  P->B = cache->batch;
+  P->cap = cache->capacity;
+  P->max_block = max_block;
+  P->max_rows = max_rows;
+  P->sms = num_sms();
+  P->chunk_keys = wl.chunk_keys;
+  P->attn_slots = wl.attn_slots;
+  P->embed = w->embed;
+  P->final_norm = w->final_norm;
+  P->lm_head = w->lm_head;
+  P->kc = (__nv_bfloat16*)cache->k;
+  P->vc = (__nv_bfloat16*)cache->v;
+  P->len = cache->len;
+  P->ws = workspace;
+  P->ws_bytes = workspace_bytes;
+  char* base = (char*)workspace;
+  P->status = (int*)(base + wl.status);
+  P->h = (float*)(base + wl.h);
+  P->xn = (__nv_bfloat16*)(base + wl.xn);
+  P->qbuf = (__nv_bfloat16*)(base + wl.qbuf);
+  P->attn = (__nv_bfloat16*)(base + wl.attn);
+  P->act = (__nv_bfloat16*)(base + wl.act);
+  P->rope = (float2*)(base + wl.rope);
+  P->amax = (unsigned long long*)(base + wl.amax);
+  P->draft_ids = (int*)(base + wl.draft_ids);
+  P->ar_ids = (int*)(base + wl.ar_ids);
+  P->gemm_part = (float*)(base + wl.gemm_part);
+  P->gemm_cnt = (int*)(base + wl.gemm_cnt);
+  P->att_o = (float*)(base + wl.att_o);
+  P->att_ml = (float2*)(base + wl.att_ml);
+  P->att_cnt = (int*)(base + wl.att_cnt);
+  P->blk_k = (__nv_bfloat16*)(base + wl.blk_k);
+  P->blk_v = (__nv_bfloat16*)(base + wl.blk_v);
+  P->layers_off = layers_off;
+  P->maps_off = maps_off;
+
+  const int D = cfg->d_model, H = cfg->n_heads, Hkv = cfg->n_kv_heads, d = cfg->head_dim, F = cfg->d_ff;
+  const int V = cfg->vocab, qkv_rows = (H + 2 * Hkv) * d;
+  bool ok = true;
+  for (int l = 0; l < L; ++l) {
+    LayerPtrs& lp = P->layer(l);
+    lp.attn_norm = w->attn_norm[l];
+    lp.mlp_norm = w->mlp_norm[l];
+    lp.q_norm = cfg->qk_norm ? w->q_norm[l] : nullptr;
+    lp.k_norm = cfg->qk_norm ? w->k_norm[l] : nullptr;
+    lp.wd_q_norm = cfg->qk_norm ? w->wd_q_norm[l] : nullptr;
+    lp.wd_k_norm = cfg->qk_norm ? w->wd_k_norm[l] : nullptr;
+    lp.w_qkv = w->w_qkv[l];
+    lp.w_o = w->w_o[l];
+    lp.w_gu = w->w_gate_up[l];
+    lp.w_down = w->w_down[l];
+    lp.wd_qkv = w->wd_qkv[l];
+    lp.wd_o = w->wd_o[l];
+    if (!lp.attn_norm || !lp.mlp_norm) ok = false;
+    if (cfg->qk_norm && (!lp.q_norm || !lp.k_norm || !lp.wd_q_norm || !lp.wd_k_norm)) ok = false;
+    ok = ok && map2d(P->lmap_mut(l, M_WQKV), lp.w_qkv, D, qkv_rows, 64, 128);
+    ok = ok && map2d(P->lmap_mut(l, M_WO), lp.w_o, H * d, D, 64, 128);
+    ok = ok && map2d(P->lmap_mut(l, M_WGU), lp.w_gu, D, 2 * F, 64, 64);
+    ok = ok && map2d(P->lmap_mut(l, M_WDOWN), lp.w_down, F, D, 64, 128);
+    ok = ok && map2d(P->lmap_mut(l, M_WDQKV), lp.wd_qkv, D, qkv_rows, 64, 128);
+    ok = ok && map2d(P->lmap_mut(l, M_WDO), lp.wd_o, H * d, D, 64, 128);
+  }
+  ok = ok && map2d(P->gmap_mut(G_LM), w->lm_head, D, V, 64, 128);
+  ok = ok && map2d(P->gmap_mut(G_XN), P->xn, D, max_rows, 64, 16);
+  ok = ok && map2d(P->gmap_mut(G_ATTN), P->attn, H * d, max_rows, 64, 16);
+  ok = ok && map2d(P->gmap_mut(G_ACT), P->act, F, max_rows, 64, 16);
+  ok = ok && map2d(P->gmap_mut(G_Q), P->qbuf, d, (uint64_t)max_rows * H + 128, 64, 128);
+  const uint64_t zc = (uint64_t)L * P->B * Hkv;
+  ok = ok && map3d(P->gmap_mut(G_KC), P->kc, d, P->cap, zc);
+  ok = ok && map3d(P->gmap_mut(G_VC), P->vc, d, P->cap, zc);
+  ok = ok && map3d(P->gmap_mut(G_KB), P->blk_k, d, max_block, zc);
+  ok = ok && map3d(P->gmap_mut(G_VB), P->blk_v, d, max_block, zc);
+  if (!ok) return ORTHRUS_ERR_ARG;
+  if (cudaMemsetAsync(workspace, 0, wl.total, (cudaStream_t)stream) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+  P->magic = kPlanMagic;
+  return ORTHRUS_OK;
+}
+
+int32_t* orthrus_status_ptr(const void* plan) {
+  const Plan* P = plan_cast(plan);
+  return P ? P->status : nullptr;
+}
+
+orthrus_status orthrus_clear_status(const void* plan, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P) return ORTHRUS_ERR_ARG;
+  return cudaMemsetAsync(P->status, 0, sizeof(int), (cudaStream_t)stream) == cudaSuccess ? ORTHRUS_OK
+                                                                                       : ORTHRUS_ERR_CUDA;
+}
+
+int32_t orthrus_decode_step_launches(const void* plan, int32_t K) {
+  const Plan* P = plan_cast(plan);
+  if (!P || K < 1 || K > P->max_block) return 0;
+  const int per_forward = 1 + 7 * P->L + 3;
+  return 2 * per_forward + 1;
+}
+
+orthrus_status orthrus_prefill(const void* plan, const int32_t* tokens, const int32_t* prompt_len, int32_t max_prompt,
+                               int32_t* pending, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !tokens || !prompt_len || !pending || max_prompt < 1) return ORTHRUS_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int b = 0; b < P->B; ++b)
+    if (prompt_len[b] < 1 || prompt_len[b] > max_prompt) return ORTHRUS_ERR_ARG;
+  for (int b = 0; b < P->B; ++b)
+    if (prompt_len[b] > P->cap) return ORTHRUS_ERR_CAPACITY;
+  const int chunk = P->max_rows;
+  for (int b = 0; b < P->B; ++b) {
+    const int Pb = prompt_len[b];
+    for (int c0 = 0; c0 < Pb; c0 += chunk) {
+      const int Q = std::min(chunk, Pb - c0);
+      const bool last = c0 + Q == Pb;
+      set_len_kernel<<<1, 1, 0, st>>>(P->len, b, c0);
+      orthrus_status s = forward(P, BLOCK_PREFILL, b, 1, Q, nullptr, nullptr, tokens, max_prompt, c0, last, true,
+                                 pending + b, nullptr, st);
+      if (s != ORTHRUS_OK) return s;
+    }
+    set_len_kernel<<<1, 1, 0, st>>>(P->len, b, Pb);
+  }
+  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
+}
+
+orthrus_status orthrus_draft_block(const void* plan, const int32_t* pending, int32_t K, int32_t* draft, float* logits,
+                                   orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !draft || K < 1 || K > P->max_block) return ORTHRUS_ERR_ARG;
+  return forward(P, BLOCK_DRAFT, 0, P->B, K, pending, nullptr, nullptr, 0, 0, true, false, draft, logits,
+                 (cudaStream_t)stream);
+}
+
+orthrus_status orthrus_verify_block(const void* plan, const int32_t* pending, const int32_t* draft, int32_t K,
+                                    int32_t* ar_argmax, float* logits, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !ar_argmax || K < 0 || K > P->max_block || (K > 0 && !draft)) return ORTHRUS_ERR_ARG;
+  return forward(P, BLOCK_VERIFY, 0, P->B, K + 1, pending, draft, nullptr, 0, 0, true, false, ar_argmax, logits,
+                 (cudaStream_t)stream);
+}
+
+orthrus_status orthrus_accept_commit(const void* plan, int32_t* pending, const int32_t* draft,
+                                     const int32_t* ar_argmax, int32_t K, int32_t* accept_len, int32_t* committed,
+                                     int32_t poison_dead, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !ar_argmax || !accept_len || !committed || K < 0 || K > P->max_block || (K > 0 && !draft))
+    return ORTHRUS_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  accept_kernel<<<P->B, 96, 0, st>>>(pending, draft, ar_argmax, K, accept_len, committed, P->len, P->status);
+  if (poison_dead)
+    poison_kernel<<<P->L * P->B * P->cfg.n_kv_heads, 128, 0, st>>>(P->kc, P->vc, P->len, accept_len, K, P->B,
+                                                                    P->cfg.n_kv_heads, P->cap, P->cfg.head_dim);
+  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
+}
+
+orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K, const int32_t* planted,
+                                   int32_t* accept_len, int32_t* committed, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !accept_len || !committed || K < 1 || K > P->max_block) return ORTHRUS_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  orthrus_status s = orthrus_draft_block(plan, pending, K, P->draft_ids, nullptr, stream);
+  if (s != ORTHRUS_OK) return s;
+  if (planted && cudaMemcpyAsync(P->draft_ids, planted, sizeof(int) * P->B * K, cudaMemcpyDeviceToDevice, st) !=
+                     cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  s = orthrus_verify_block(plan, pending, P->draft_ids, K, P->ar_ids, nullptr, stream);
+  if (s != ORTHRUS_OK) return s;
+  return orthrus_accept_commit(plan, pending, P->draft_ids, P->ar_ids, K, accept_len, committed, 0, stream);
+}
+
+// ---- single kernels -------------------------------------------------------
+
+size_t orthrus_attention_workspace_bytes(int32_t batch, int32_t n_kv_heads, int32_t group, int32_t Q, int32_t head_dim,
+                                         int32_t capacity) {
+  if (batch < 1 || n_kv_heads < 1 || group < 1 || Q < 1 || capacity < 1 || (head_dim != 64 && head_dim != 128))
+    return 0;
+  const int rt = (Q * group + 127) / 128;
+  const int ck = attn_chunk_keys(batch, n_kv_heads, rt, capacity);
+  const size_t chunks = (capacity + ck - 1) / ck + 1;
+  const size_t slots = (size_t)batch * n_kv_heads * rt;
+  return align_up(slots * chunks * 128 * head_dim * 4, 256) + align_up(slots * chunks * 128 * 8, 256) +
+         align_up(slots * 4, 256);
+}
+
+orthrus_status orthrus_attention(const void* q, const void* k_cache, const void* v_cache, const void* k_blk,
+                                 const void* v_blk, const int32_t* len, int32_t batch, int32_t n_kv_heads,
+                                 int32_t group, int32_t Q, int32_t head_dim, int32_t capacity, int32_t blk_stride,
+                                 int32_t mode, void* out, void* workspace, size_t workspace_bytes, int32_t* status,
+                                 orthrus_stream stream) {
+  if (!q || !k_cache || !v_cache || !len || !out || !workspace || (mode != 0 && mode != 1)) return ORTHRUS_ERR_ARG;
+  if (mode == 0 && (!k_blk || !v_blk || blk_stride < Q)) return ORTHRUS_ERR_ARG;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return ORTHRUS_ERR_UNSUPPORTED;
+  if (Q > 64 && mode == 0) return ORTHRUS_ERR_UNSUPPORTED;
+  const size_t need = orthrus_attention_workspace_bytes(batch, n_kv_heads, group, Q, head_dim, capacity);
+  if (!need) return ORTHRUS_ERR_ARG;
+  if (workspace_bytes < need) return ORTHRUS_ERR_WORKSPACE;
+  if (!encode_fn()) return ORTHRUS_ERR_CUDA;
+  const int rt = (Q * group + 127) / 128;
+  const int ck = attn_chunk_keys(batch, n_kv_heads, rt, capacity);
+  const int chunks = (capacity + ck - 1) / ck + 1;
+  const size_t slots = (size_t)batch * n_kv_heads * rt;
+  char* base = (char*)workspace;
+  float* part_o = (float*)base;
+  float2* part_ml = (float2*)(base + align_up(slots * chunks * 128 * head_dim * 4, 256));
+  int* counter = (int*)(base + align_up(slots * chunks * 128 * head_dim * 4, 256) + align_up(slots * chunks * 128 * 8, 256));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(counter, 0, slots * 4, st) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+  CUtensorMap tq, tk, tv, tkb, tvb;
+  const uint64_t z = (uint64_t)batch * n_kv_heads;
+  bool ok = map2d(&tq, q, head_dim, z * Q * group, 64, 128);
+  ok = ok && map3d(&tk, k_cache, head_dim, capacity, z) && map3d(&tv, v_cache, head_dim, capacity, z);
+  if (mode == 0) ok = ok && map3d(&tkb, k_blk, head_dim, blk_stride, z) && map3d(&tvb, v_blk, head_dim, blk_stride, z);
+  else {
+    tkb = tk;
+    tvb = tv;
+  }
+  if (!ok) return ORTHRUS_ERR_ARG;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = batch;
+  a.Hkv = n_kv_heads;
+  a.G = group;
+  a.Q = Q;
+  a.d = head_dim;
+  a.mode = mode;
+  a.b0 = 0;
+  a.rows = Q * group;
+  a.row_tiles = rt;
+  a.chunk_keys = ck;
+  a.cap = capacity;
+  a.z_cache = 0;
+  a.z_blk = 0;
+  a.max_chunks = (capacity + ck - 1) / ck + (mode == 0 ? 1 : 0);
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
+  a.len = len;
+  a.out = (__nv_bfloat16*)out;
+  a.part_o = part_o;
+  a.part_ml = part_ml;
+  a.counter = counter;
+  a.status = status;
+  return launch_attention(head_dim, tq, tk, tv, tkb, tvb, a, st) == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
+}
+
+size_t orthrus_linear_workspace_bytes(int32_t M, int32_t N, int32_t Kd) {
+  if (M < 1 || N < 128 || N % 128 || Kd < 64 || Kd % 64) return 0;
+  const size_t tiles = (size_t)((M + 127) / 128) * (N / 128);
+  return align_up((size_t)2 * num_sms() * 128 * 128 * 4, 256) + align_up(tiles * 4, 256);
+}
+
+orthrus_status orthrus_linear(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t Kd,
+                              void* workspace, size_t workspace_bytes, int32_t* status, orthrus_stream stream) {
+  if (!X || !W || !Y || !workspace) return ORTHRUS_ERR_ARG;
+  const size_t need = orthrus_linear_workspace_bytes(M, N, Kd);
+  if (!need) return ORTHRUS_ERR_UNSUPPORTED;
+  if (workspace_bytes < need) return ORTHRUS_ERR_WORKSPACE;
+  if (!encode_fn()) return ORTHRUS_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = (char*)workspace;
+  const size_t part_bytes = align_up((size_t)2 * num_sms() * 128 * 128 * 4, 256);
+  int* cnt = (int*)(base + part_bytes);
+  const size_t tiles = (size_t)((M + 127) / 128) * (N / 128);
+  if (cudaMemsetAsync(cnt, 0, tiles * 4, st) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+  CUtensorMap tw, tx;
+  if (!map2d(&tw, W, Kd, N, 64, 128) || !map2d(&tx, X, Kd, M, 64, 16)) return ORTHRUS_ERR_ARG;
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.partial = (float*)base;
+  a.tile_counter = cnt;
+  a.status = status;
+  a.out_f32 = Y;
+  a.ld_out = N;
+  return launch_gemm<EPI_STORE>(tw, tx, a, N, Kd, M, st) == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -27,7 +27,7 @@ import numpy as np
 __all__ = [
     "ModelShape", "TINY", "TINY_QK", "QWEN3_8B", "tensor_specs", "make_weights",
     "make_prompt", "round_to_bf16_bits", "bf16_bits_to_f32", "planted_accepts",
-    "planted_drafts", "uniform_tokens",
+    "planted_drafts", "uniform_tokens", "normal_bf16",
 ]
 
 
@@ -146,6 +146,13 @@ def make_weights(shape: ModelShape, seed_base: int, seed_draft: int, std: float 
             _normal_bf16(seed_base if kind == "base" else seed_draft, idx, n, std, buf, pool)
             out[name] = buf.reshape(dims)
     return out
+
+
+def normal_bf16(shape, seed: int, std: float = 1.0) -> np.ndarray:
+    """N(0, std) float32 rounded to bfloat16; uint16 bit patterns of the given shape."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(0xB16,))))
+    a = g.standard_normal(int(np.prod(shape)), dtype=np.float32) * np.float32(std)
+    return round_to_bf16_bits(a).reshape(shape)
 
 
 def uniform_tokens(vocab: int, n: int, seed: int) -> np.ndarray:

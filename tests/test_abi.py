@@ -1,0 +1,79 @@
+"""The C-ABI library loads and exports every entry point include/orthrus.h
+declares; host-only size queries and argument checks work without a GPU."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import synth
+from shared_kv_draft_b200 import orthrus
+from shared_kv_draft_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return orthrus.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "orthrus.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(orthrus_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(n for n, _, _ in orthrus.SIGNATURES) == names
+
+
+def test_core_calls_declared():
+    names = declared_symbols()
+    for n in ("orthrus_draft_block", "orthrus_verify_block", "orthrus_accept_commit", "orthrus_decode_step"):
+        assert n in names
+
+
+def test_block_scratch_is_four_and_a_half_mib(lib):
+    cfg = orthrus.make_config(synth.QWEN3_8B)
+    assert orthrus.block_scratch_bytes(cfg, 1, 32) == 4_718_592
+
+
+def test_size_queries_reject_bad_shapes(lib):
+    cfg = orthrus.make_config(synth.QWEN3_8B)
+    assert orthrus.plan_bytes(cfg) > 0
+    assert orthrus.workspace_bytes(cfg, 1, 2048, 32, 33) > 0
+    assert orthrus.workspace_bytes(cfg, 1, 2048, 65, 66 * 1) == 0      # K > 64
+    assert orthrus.workspace_bytes(cfg, 2, 2048, 32, 33) == 0          # rows < batch*(K+1)
+    bad = orthrus.make_config(synth.QWEN3_8B)
+    bad.head_dim = 96
+    assert orthrus.plan_bytes(bad) == 0
+    bad = orthrus.make_config(synth.QWEN3_8B)
+    bad.vocab = 1000
+    assert orthrus.plan_bytes(bad) == 0
+    off = orthrus.block_scratch_offset(cfg, 1, 2048, 32, 33)
+    assert 0 < off < orthrus.workspace_bytes(cfg, 1, 2048, 32, 33)
+
+
+def test_null_plan_is_rejected(lib):
+    assert lib.orthrus_decode_step(None, None, 32, None, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_draft_block(None, None, 4, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_decode_step_launches(None, 4) == 0
+    buf = C.create_string_buffer(64)  # not an initialised plan
+    assert lib.orthrus_verify_block(buf, None, None, 4, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_status_ptr(buf) is None
+
+
+def test_plan_init_rejects_nulls(lib):
+    cfg = orthrus.make_config(synth.TINY)
+    n = orthrus.plan_bytes(cfg)
+    buf = C.create_string_buffer(n)
+    w = orthrus.Weights()
+    cache = orthrus.Cache(None, None, None, 1, 64)
+    code = lib.orthrus_plan_init(buf, n, C.byref(cfg), C.byref(w), C.byref(cache), 4, 5, None, 0, None)
+    assert code == orthrus.ERR_ARG
