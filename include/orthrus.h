@@ -144,6 +144,31 @@ orthrus_status orthrus_clear_status(const void* plan, orthrus_stream stream);
  * (planted drafts add one device-to-device copy, not a kernel). */
 int32_t orthrus_decode_step_launches(const void* plan, int32_t K);
 
+/* Kernel kinds reported by orthrus_trace. */
+enum {
+  ORTHRUS_KIND_EMBED = 0,      /* block embedding + RoPE table + capacity check   */
+  ORTHRUS_KIND_RMSNORM = 1,    /* RMSNorm to bf16                                  */
+  ORTHRUS_KIND_GEMM_QKV = 2,   /* q/k/v projection + QK-norm + RoPE + K/V store   */
+  ORTHRUS_KIND_ATTENTION = 3,  /* block attention                                  */
+  ORTHRUS_KIND_GEMM_O = 4,     /* output projection + residual                     */
+  ORTHRUS_KIND_GEMM_GATE_UP = 5, /* gate/up projection + SwiGLU                    */
+  ORTHRUS_KIND_GEMM_DOWN = 6,  /* down projection + residual                       */
+  ORTHRUS_KIND_LM_HEAD = 7,    /* LM head + running argmax                         */
+  ORTHRUS_KIND_ARGMAX = 8,     /* argmax finalisation                              */
+  ORTHRUS_KIND_ACCEPT = 9,     /* greedy consensus + KV commit                     */
+  ORTHRUS_KIND_OTHER = 10,     /* poisoning, length updates, planted-draft copy    */
+  ORTHRUS_KIND_END = 11        /* marker after the last launch of a call          */
+};
+
+/* Profiling hook. While set, every launch made by the calls below is preceded
+ * by cudaEventRecord(events[i], stream) with kinds[i] = its ORTHRUS_KIND_*, and
+ * each call ends with an ORTHRUS_KIND_END marker; *count holds the number of
+ * events used (recording stops at `capacity`). events are cudaEvent_t handles
+ * created by the caller with timing enabled; launch i lasted
+ * elapsed(events[i], events[i+1]). Pass events == NULL to switch it off.
+ * Host memory of `kinds` and `count` must stay valid while the hook is set. */
+orthrus_status orthrus_trace(void* plan, void* const* events, int32_t* kinds, int32_t capacity, int32_t* count);
+
 /* ---- the decode step ---------------------------------------------------- */
 
 /* AR prefill (atlas summary "Approach": the frozen backbone does prefill and

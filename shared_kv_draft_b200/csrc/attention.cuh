@@ -81,6 +81,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int bh = blockIdx.z;  // local sequence * Hkv + kvh
   const int bb = bh / a.Hkv, kvh = bh - bb * a.Hkv;
   const int b = a.b0 + bb;
+  griddep_wait();  // q, the cache and len come from earlier kernels
+  griddep_launch();
   const int n = a.len[b];
 
   // ---- key range of this CTA ------------------------------------------------

@@ -53,7 +53,7 @@ struct GemmArgs {
   long long total_units;
   int stages;
   int swiglu_F;              // SwiGLU: row offset of the up rows in W
-  float* partial;            // [2 * grid][128 * 128]
+  float* partial;            // [2 * grid][128 rows][Mt] fp32 partial sums of split tiles
   int* tile_counter;         // [m_tiles * n_tiles], zero between launches
   int* status;
   float* out_f32;            // STORE: Y[M][ld_out]; RESID: h[M][ld_out] (+=)
@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_launch();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -266,22 +267,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t pol_x = policy_evict_last();
       int issued[16];
       for (int s = 0; s < 16; ++s) issued[s] = -1;
-      int it = 0;
-      for (long long u = u0; u < u1; ++u, ++it) {
+      auto load_w = [&](int s, long long u) {
         const int t = (int)(u / kc), k = (int)(u - (long long)t * kc);
-        const int nt = t / a.m_tiles, mt = t - nt * a.m_tiles;
-        const int s = it % S, ph = (it / S) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, a.status)) break;
+        const int nt = t / a.m_tiles;
         uint8_t* wdst = smem + (size_t)s * stage_bytes;
-        uint8_t* xdst = wdst + 16384;
-        mbar_arrive_expect_tx(&full[s], stage_bytes);
         if constexpr (EPI == EPI_SWIGLU) {
           tma_load_2d_hint(wdst, &tmW, &full[s], k * 64, nt * 64, pol_w);
           tma_load_2d_hint(wdst + 8192, &tmW, &full[s], k * 64, a.swiglu_F + nt * 64, pol_w);
         } else {
           tma_load_2d_hint(wdst, &tmW, &full[s], k * 64, nt * 128, pol_w);
         }
-        for (int r = 0; r < a.Mt; r += 16) tma_load_2d_hint(xdst + r * 128, &tmX, &full[s], k * 64, mt * 128 + r, pol_x);
+      };
+      auto load_x = [&](int s, long long u) {
+        const int t = (int)(u / kc), k = (int)(u - (long long)t * kc);
+        const int mt = t - (t / a.m_tiles) * a.m_tiles;
+        uint8_t* xdst = smem + (size_t)s * stage_bytes + 16384;
+        tma_load_2d_hint(xdst, &tmX, &full[s], k * 64, mt * 128, pol_x);  // one box of Mt token rows
+      };
+      // weights never depend on earlier kernels: fill the ring with weight tiles
+      // before waiting for the predecessor, then add the activation tiles
+      const int pre = (int)min((long long)S, u1 - u0);
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], stage_bytes);
+        load_w(i, u0 + i);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) {
+        load_x(i, u0 + i);
+        issued[i] = 0;
+      }
+      int it = pre;
+      for (long long u = u0 + pre; u < u1; ++u, ++it) {
+        const int s = it % S, ph = (it / S) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, a.status)) break;
+        mbar_arrive_expect_tx(&full[s], stage_bytes);
+        load_w(s, u);
+        load_x(s, u);
         issued[s] = ph;
       }
       // every load issued must have landed before the CTA may exit
@@ -327,6 +348,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ---------------- epilogue warps ----------------
+    griddep_wait();  // outputs and shared scratch are touched only after the predecessor finished
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     int seg = 0;
@@ -360,13 +382,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) mbar_arrive(&acce[buf]);
       } else {
         // write this CTA's partial sum of the tile, then count arrivals
+        // this thread's Mt partial sums, contiguous: [slot][row][Mt]
         const int slot = 2 * c + (t == first_tile ? 0 : 1);
-        float* part = a.partial + (size_t)slot * (128 * 128);
+        float* part = a.partial + (size_t)slot * (128 * 128) + (size_t)row * a.Mt;
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
           tmem_ld32(taddr + m0, v);
+          const int n4 = min(32, a.Mt - m0) / 4;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (m0 + j < m_valid) part[(m0 + j) * 128 + row] = v[j];
+          for (int q = 0; q < 8; ++q)
+            if (q < n4) __stcg(reinterpret_cast<float4*>(part + m0) + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
         }
         tc_fence_before();
         __syncwarp();
@@ -384,14 +408,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __threadfence();
           if (threadIdx.x == 64) a.tile_counter[t] = 0;
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+            const int n4 = min(32, a.Mt - m0) / 4;
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
+            for (int cc = c_lo; cc <= c_hi; ++cc) {  // fixed k order: the sum does not depend on arrival order
               const int ft = (int)(unit_start(W, G, cc) / kc);
-              const float* pp = a.partial + (size_t)(2 * cc + (t == ft ? 0 : 1)) * (128 * 128);
+              const float4* pp = reinterpret_cast<const float4*>(
+                  a.partial + (size_t)(2 * cc + (t == ft ? 0 : 1)) * (128 * 128) + (size_t)row * a.Mt + m0);
+              float4 x[8];
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (m0 + j < m_valid) v[j] += __ldcg(pp + (m0 + j) * 128 + row);
+              for (int q = 0; q < 8; ++q) x[q] = q < n4 ? __ldcg(pp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                v[4 * q] += x[q].x;
+                v[4 * q + 1] += x[q].y;
+                v[4 * q + 2] += x[q].z;
+                v[4 * q + 3] += x[q].w;
+              }
             }
             epilogue_group<EPI>(a, v, row, m0, mt, nt, m_valid, epi, red);
           }

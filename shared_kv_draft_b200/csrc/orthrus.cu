@@ -3,10 +3,12 @@
 // passes, and the C-ABI entry points declared in include/orthrus.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
 #include <cmath>
+#include <utility>
 
 #include "attention.cuh"
 #include "gemm.cuh"
@@ -82,12 +84,41 @@ int num_sms() {
 
 constexpr size_t kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100
 
+// Programmatic dependent launch for every kernel (ORTHRUS_PDL=0 in the
+// environment turns it off): a kernel may begin its prologue and weight loads
+// while its predecessor drains; its griddepcontrol.wait orders everything else.
+bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("ORTHRUS_PDL");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // plan
 // ---------------------------------------------------------------------------
 constexpr uint64_t kPlanMagic = 0x4F52544852555331ull;  // "ORTHRUS1"
 enum { M_WQKV = 0, M_WO, M_WGU, M_WDOWN, M_WDQKV, M_WDO, M_PER_LAYER };
-enum { G_LM = 0, G_XN, G_ATTN, G_ACT, G_Q, G_KC, G_VC, G_KB, G_VB, G_COUNT };
+// activation maps exist for every token-tile height Mt = 16, 32, ..., 128 (index Mt/16 - 1)
+enum { G_LM = 0, G_Q, G_KC, G_VC, G_KB, G_VB, G_XN, G_ATTN = G_XN + 8, G_ACT = G_ATTN + 8, G_COUNT = G_ACT + 8 };
 
 struct LayerPtrs {
   const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
@@ -117,6 +148,11 @@ struct alignas(64) Plan {
   float2* att_ml;
   int* att_cnt;
   size_t layers_off, maps_off;
+  // profiling hook (host memory, written during the calls)
+  void* const* trace_ev;
+  int32_t* trace_kind;
+  int32_t trace_cap;
+  int32_t* trace_count;
 
   const LayerPtrs& layer(int l) const { return reinterpret_cast<const LayerPtrs*>((const char*)this + layers_off)[l]; }
   LayerPtrs& layer(int l) { return reinterpret_cast<LayerPtrs*>((char*)this + layers_off)[l]; }
@@ -185,8 +221,12 @@ int gemm_counter_count(const orthrus_config* c, int max_rows) {
   return mt * nt;
 }
 
-WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows, int cap) {
+// Rows allocated for activation buffers: a multiple of 128 so that any token tile fits.
+int act_rows(int max_rows) { return round_up(std::max(max_rows, 128), 128); }
+
+WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows_req, int cap) {
   WsLayout w{};
+  const int max_rows = act_rows(max_rows_req);
   const int D = c->d_model, Hd = c->n_heads * c->head_dim, F = c->d_ff, d = c->head_dim, L = c->n_layers;
   const int G = c->n_heads / c->n_kv_heads, Hkv = c->n_kv_heads;
   const int sms = num_sms();
@@ -194,7 +234,7 @@ WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows, 
   const int ck = attn_chunk_keys(B, Hkv, rt_dec, cap);
   w.chunk_keys = ck;
   const int max_chunks = (cap + ck - 1) / ck + 1;
-  const int rt_pre = (G * max_rows + 127) / 128;
+  const int rt_pre = (G * max_rows_req + 127) / 128;
   w.attn_slots = std::max(B * Hkv * rt_dec, Hkv * rt_pre) * max_chunks;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -251,8 +291,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs
   const size_t smem = gemm_smem_bytes(a.Mt, a.stages);
   static bool attr = false;
   if (!attr) attr = set_smem_attr(gemm_kernel<EPI>, kSmemLimit);
-  gemm_kernel<EPI><<<G, kGemmThreads, smem, st>>>(tmW, tmX, a);
-  return cudaGetLastError();
+  return launch(gemm_kernel<EPI>, dim3(G), dim3(kGemmThreads), smem, st, tmW, tmX, a);
 }
 
 cudaError_t launch_attention(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -262,13 +301,27 @@ cudaError_t launch_attention(int d, const CUtensorMap& tq, const CUtensorMap& tk
   if (d == 128) {
     static bool attr = false;
     if (!attr) attr = set_smem_attr(attention_kernel<128>, kSmemLimit);
-    attention_kernel<128><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, tkb, tvb, a);
+    return launch(attention_kernel<128>, grid, dim3(kAttnThreads), smem, st, tq, tk, tv, tkb, tvb, a);
   } else {
     static bool attr = false;
     if (!attr) attr = set_smem_attr(attention_kernel<64>, kSmemLimit);
-    attention_kernel<64><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, tkb, tvb, a);
+    return launch(attention_kernel<64>, grid, dim3(kAttnThreads), smem, st, tq, tk, tv, tkb, tvb, a);
   }
-  return cudaGetLastError();
+}
+
+void mark(const Plan* P, int kind, cudaStream_t st) {
+  if (!P->trace_ev || !P->trace_count) return;
+  const int i = *P->trace_count;
+  if (i >= P->trace_cap) return;
+  cudaEventRecord((cudaEvent_t)P->trace_ev[i], st);
+  P->trace_kind[i] = kind;
+  *P->trace_count = i + 1;
+}
+
+// token-tile height of a GEMM over M rows (must match launch_gemm) -> map index
+int mt_index(int M) {
+  const int Mt = M > 128 ? 128 : round_up(std::max(M, 1), 16);
+  return Mt / 16 - 1;
 }
 
 GemmArgs base_gemm_args(const Plan* P) {
@@ -291,7 +344,6 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
   const int D = c.d_model, H = c.n_heads, Hkv = c.n_kv_heads, d = c.head_dim, F = c.d_ff, V = c.vocab;
   const int G = H / Hkv, M = nb * Q;
   const bool draft_view = kind == BLOCK_DRAFT;
-  cudaError_t e;
 
   EmbedArgs ea;
   ea.kind = kind;
@@ -314,7 +366,8 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
   ea.h = P->h;
   ea.rope = P->rope;
   ea.status = P->status;
-  embed_kernel<<<M, 256, 0, st>>>(ea);
+  mark(P, ORTHRUS_KIND_EMBED, st);
+  if (launch(embed_kernel, dim3(M), dim3(256), 0, st, ea) != cudaSuccess) return ORTHRUS_ERR_CUDA;
 
   AttnArgs aa;
   memset(&aa, 0, sizeof(aa));
@@ -341,7 +394,10 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
 
   for (int l = 0; l < P->L; ++l) {
     const LayerPtrs& lp = P->layer(l);
-    rmsnorm_kernel<<<M, 256, 0, st>>>(P->h, D, lp.attn_norm, c.rms_eps, P->xn, 0, 1, nullptr);
+    mark(P, ORTHRUS_KIND_RMSNORM, st);
+    if (launch(rmsnorm_kernel, dim3(M), dim3(256), 0, st, (const float*)P->h, D, lp.attn_norm, c.rms_eps, P->xn, 0, 1,
+               (unsigned long long*)nullptr) != cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
 
     GemmArgs g = base_gemm_args(P);
     g.qkv.H = H;
@@ -369,49 +425,63 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
       g.qkv.kv_stride = P->cap;
     }
     const int qkv_rows = (H + 2 * Hkv) * d;
-    if ((e = launch_gemm<EPI_QKV>(P->lmap(l, draft_view ? M_WDQKV : M_WQKV), P->gmap(G_XN), g, qkv_rows, D, M, st)) !=
+    mark(P, ORTHRUS_KIND_GEMM_QKV, st);
+    if ((launch_gemm<EPI_QKV>(P->lmap(l, draft_view ? M_WDQKV : M_WQKV), P->gmap(G_XN + mt_index(M)), g, qkv_rows, D, M, st)) !=
         cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
     aa.z_cache = l * P->B * Hkv;
     aa.z_blk = l * P->B * Hkv;
-    if ((e = launch_attention(d, P->gmap(G_Q), P->gmap(G_KC), P->gmap(G_VC), P->gmap(G_KB), P->gmap(G_VB), aa, st)) !=
+    mark(P, ORTHRUS_KIND_ATTENTION, st);
+    if ((launch_attention(d, P->gmap(G_Q), P->gmap(G_KC), P->gmap(G_VC), P->gmap(G_KB), P->gmap(G_VB), aa, st)) !=
         cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
     g = base_gemm_args(P);
     g.out_f32 = P->h;
     g.ld_out = D;
-    if ((e = launch_gemm<EPI_RESID>(P->lmap(l, draft_view ? M_WDO : M_WO), P->gmap(G_ATTN), g, D, H * d, M, st)) !=
+    mark(P, ORTHRUS_KIND_GEMM_O, st);
+    if ((launch_gemm<EPI_RESID>(P->lmap(l, draft_view ? M_WDO : M_WO), P->gmap(G_ATTN + mt_index(M)), g, D, H * d, M, st)) !=
         cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
-    rmsnorm_kernel<<<M, 256, 0, st>>>(P->h, D, lp.mlp_norm, c.rms_eps, P->xn, 0, 1, nullptr);
+    mark(P, ORTHRUS_KIND_RMSNORM, st);
+    if (launch(rmsnorm_kernel, dim3(M), dim3(256), 0, st, (const float*)P->h, D, lp.mlp_norm, c.rms_eps, P->xn, 0, 1,
+               (unsigned long long*)nullptr) != cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
     g = base_gemm_args(P);
     g.out_bf16 = P->act;
     g.ld_out = F;
     g.swiglu_F = F;
-    if ((e = launch_gemm<EPI_SWIGLU>(P->lmap(l, M_WGU), P->gmap(G_XN), g, 2 * F, D, M, st)) != cudaSuccess)
+    mark(P, ORTHRUS_KIND_GEMM_GATE_UP, st);
+    if ((launch_gemm<EPI_SWIGLU>(P->lmap(l, M_WGU), P->gmap(G_XN + mt_index(M)), g, 2 * F, D, M, st)) != cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
     g = base_gemm_args(P);
     g.out_f32 = P->h;
     g.ld_out = D;
-    if ((e = launch_gemm<EPI_RESID>(P->lmap(l, M_WDOWN), P->gmap(G_ACT), g, D, F, M, st)) != cudaSuccess)
+    mark(P, ORTHRUS_KIND_GEMM_DOWN, st);
+    if ((launch_gemm<EPI_RESID>(P->lmap(l, M_WDOWN), P->gmap(G_ACT + mt_index(M)), g, D, F, M, st)) != cudaSuccess)
       return ORTHRUS_ERR_CUDA;
   }
 
   if (!head) return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
   const int HR = last_row_only ? nb : M;
-  rmsnorm_kernel<<<HR, 256, 0, st>>>(P->h, D, P->final_norm, c.rms_eps, P->xn, last_row_only ? Q - 1 : 0,
-                                     last_row_only ? Q : 1, P->amax);
+  mark(P, ORTHRUS_KIND_RMSNORM, st);
+  if (launch(rmsnorm_kernel, dim3(HR), dim3(256), 0, st, (const float*)P->h, D, P->final_norm, c.rms_eps, P->xn,
+             last_row_only ? Q - 1 : 0, last_row_only ? Q : 1, P->amax) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
   GemmArgs g = base_gemm_args(P);
   g.amax = P->amax;
   g.logits = logits;
   g.ld_logits = V;
-  if ((e = launch_gemm<EPI_ARGMAX>(P->gmap(G_LM), P->gmap(G_XN), g, V, D, HR, st)) != cudaSuccess)
+  mark(P, ORTHRUS_KIND_LM_HEAD, st);
+  if ((launch_gemm<EPI_ARGMAX>(P->gmap(G_LM), P->gmap(G_XN + mt_index(HR)), g, V, D, HR, st)) != cudaSuccess)
     return ORTHRUS_ERR_CUDA;
-  argmax_finalize_kernel<<<(HR + 127) / 128, 128, 0, st>>>(P->amax, HR, argmax_out, P->status);
+  mark(P, ORTHRUS_KIND_ARGMAX, st);
+  if (launch(argmax_finalize_kernel, dim3((HR + 127) / 128), dim3(128), 0, st, (const unsigned long long*)P->amax, HR,
+             argmax_out, P->status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }
 
@@ -535,10 +605,13 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
     ok = ok && map2d(P->lmap_mut(l, M_WDO), lp.wd_o, H * d, D, 64, 128);
   }
   ok = ok && map2d(P->gmap_mut(G_LM), w->lm_head, D, V, 64, 128);
-  ok = ok && map2d(P->gmap_mut(G_XN), P->xn, D, max_rows, 64, 16);
-  ok = ok && map2d(P->gmap_mut(G_ATTN), P->attn, H * d, max_rows, 64, 16);
-  ok = ok && map2d(P->gmap_mut(G_ACT), P->act, F, max_rows, 64, 16);
-  ok = ok && map2d(P->gmap_mut(G_Q), P->qbuf, d, (uint64_t)max_rows * H + 128, 64, 128);
+  const int rows = act_rows(max_rows);
+  for (int i = 0; i < 8; ++i) {
+    ok = ok && map2d(P->gmap_mut(G_XN + i), P->xn, D, rows, 64, 16 * (i + 1));
+    ok = ok && map2d(P->gmap_mut(G_ATTN + i), P->attn, H * d, rows, 64, 16 * (i + 1));
+    ok = ok && map2d(P->gmap_mut(G_ACT + i), P->act, F, rows, 64, 16 * (i + 1));
+  }
+  ok = ok && map2d(P->gmap_mut(G_Q), P->qbuf, d, (uint64_t)rows * H + 128, 64, 128);
   const uint64_t zc = (uint64_t)L * P->B * Hkv;
   ok = ok && map3d(P->gmap_mut(G_KC), P->kc, d, P->cap, zc);
   ok = ok && map3d(P->gmap_mut(G_VC), P->vc, d, P->cap, zc);
@@ -560,6 +633,24 @@ orthrus_status orthrus_clear_status(const void* plan, orthrus_stream stream) {
   if (!P) return ORTHRUS_ERR_ARG;
   return cudaMemsetAsync(P->status, 0, sizeof(int), (cudaStream_t)stream) == cudaSuccess ? ORTHRUS_OK
                                                                                        : ORTHRUS_ERR_CUDA;
+}
+
+orthrus_status orthrus_trace(void* plan, void* const* events, int32_t* kinds, int32_t capacity, int32_t* count) {
+  Plan* P = plan_cast(plan);
+  if (!P) return ORTHRUS_ERR_ARG;
+  if (!events) {
+    P->trace_ev = nullptr;
+    P->trace_kind = nullptr;
+    P->trace_count = nullptr;
+    P->trace_cap = 0;
+    return ORTHRUS_OK;
+  }
+  if (!kinds || !count || capacity < 1) return ORTHRUS_ERR_ARG;
+  P->trace_ev = events;
+  P->trace_kind = kinds;
+  P->trace_cap = capacity;
+  P->trace_count = count;
+  return ORTHRUS_OK;
 }
 
 int32_t orthrus_decode_step_launches(const void* plan, int32_t K) {
@@ -584,13 +675,16 @@ orthrus_status orthrus_prefill(const void* plan, const int32_t* tokens, const in
     for (int c0 = 0; c0 < Pb; c0 += chunk) {
       const int Q = std::min(chunk, Pb - c0);
       const bool last = c0 + Q == Pb;
-      set_len_kernel<<<1, 1, 0, st>>>(P->len, b, c0);
+      mark(P, ORTHRUS_KIND_OTHER, st);
+      if (launch(set_len_kernel, dim3(1), dim3(1), 0, st, P->len, b, c0) != cudaSuccess) return ORTHRUS_ERR_CUDA;
       orthrus_status s = forward(P, BLOCK_PREFILL, b, 1, Q, nullptr, nullptr, tokens, max_prompt, c0, last, true,
                                  pending + b, nullptr, st);
       if (s != ORTHRUS_OK) return s;
     }
-    set_len_kernel<<<1, 1, 0, st>>>(P->len, b, Pb);
+    mark(P, ORTHRUS_KIND_OTHER, st);
+    if (launch(set_len_kernel, dim3(1), dim3(1), 0, st, P->len, b, Pb) != cudaSuccess) return ORTHRUS_ERR_CUDA;
   }
+  mark(P, ORTHRUS_KIND_END, st);
   return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }
 
@@ -598,16 +692,20 @@ orthrus_status orthrus_draft_block(const void* plan, const int32_t* pending, int
                                    orthrus_stream stream) {
   const Plan* P = plan_cast(plan);
   if (!P || !pending || !draft || K < 1 || K > P->max_block) return ORTHRUS_ERR_ARG;
-  return forward(P, BLOCK_DRAFT, 0, P->B, K, pending, nullptr, nullptr, 0, 0, true, false, draft, logits,
-                 (cudaStream_t)stream);
+  orthrus_status s = forward(P, BLOCK_DRAFT, 0, P->B, K, pending, nullptr, nullptr, 0, 0, true, false, draft, logits,
+                             (cudaStream_t)stream);
+  mark(P, ORTHRUS_KIND_END, (cudaStream_t)stream);
+  return s;
 }
 
 orthrus_status orthrus_verify_block(const void* plan, const int32_t* pending, const int32_t* draft, int32_t K,
                                     int32_t* ar_argmax, float* logits, orthrus_stream stream) {
   const Plan* P = plan_cast(plan);
   if (!P || !pending || !ar_argmax || K < 0 || K > P->max_block || (K > 0 && !draft)) return ORTHRUS_ERR_ARG;
-  return forward(P, BLOCK_VERIFY, 0, P->B, K + 1, pending, draft, nullptr, 0, 0, true, false, ar_argmax, logits,
-                 (cudaStream_t)stream);
+  orthrus_status s = forward(P, BLOCK_VERIFY, 0, P->B, K + 1, pending, draft, nullptr, 0, 0, true, false, ar_argmax,
+                             logits, (cudaStream_t)stream);
+  mark(P, ORTHRUS_KIND_END, (cudaStream_t)stream);
+  return s;
 }
 
 orthrus_status orthrus_accept_commit(const void* plan, int32_t* pending, const int32_t* draft,
@@ -617,10 +715,17 @@ orthrus_status orthrus_accept_commit(const void* plan, int32_t* pending, const i
   if (!P || !pending || !ar_argmax || !accept_len || !committed || K < 0 || K > P->max_block || (K > 0 && !draft))
     return ORTHRUS_ERR_ARG;
   cudaStream_t st = (cudaStream_t)stream;
-  accept_kernel<<<P->B, 96, 0, st>>>(pending, draft, ar_argmax, K, accept_len, committed, P->len, P->status);
+  mark(P, ORTHRUS_KIND_ACCEPT, st);
+  if (launch(accept_kernel, dim3(P->B), dim3(96), 0, st, pending, draft, ar_argmax, K, accept_len, committed, P->len,
+             (const int*)P->status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  if (poison_dead) mark(P, ORTHRUS_KIND_OTHER, st);
   if (poison_dead)
-    poison_kernel<<<P->L * P->B * P->cfg.n_kv_heads, 128, 0, st>>>(P->kc, P->vc, P->len, accept_len, K, P->B,
-                                                                    P->cfg.n_kv_heads, P->cap, P->cfg.head_dim);
+    if (launch(poison_kernel, dim3(P->L * P->B * P->cfg.n_kv_heads), dim3(128), 0, st, P->kc, P->vc,
+               (const int*)P->len, (const int*)accept_len, K, P->B, P->cfg.n_kv_heads, P->cap, P->cfg.head_dim) !=
+        cudaSuccess)
+      return ORTHRUS_ERR_CUDA;
+  mark(P, ORTHRUS_KIND_END, st);
   return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }
 
@@ -631,6 +736,7 @@ orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K
   cudaStream_t st = (cudaStream_t)stream;
   orthrus_status s = orthrus_draft_block(plan, pending, K, P->draft_ids, nullptr, stream);
   if (s != ORTHRUS_OK) return s;
+  if (planted) mark(P, ORTHRUS_KIND_OTHER, st);
   if (planted && cudaMemcpyAsync(P->draft_ids, planted, sizeof(int) * P->B * K, cudaMemcpyDeviceToDevice, st) !=
                      cudaSuccess)
     return ORTHRUS_ERR_CUDA;
@@ -732,7 +838,7 @@ orthrus_status orthrus_linear(const void* X, const void* W, float* Y, int32_t M,
   const size_t tiles = (size_t)((M + 127) / 128) * (N / 128);
   if (cudaMemsetAsync(cnt, 0, tiles * 4, st) != cudaSuccess) return ORTHRUS_ERR_CUDA;
   CUtensorMap tw, tx;
-  if (!map2d(&tw, W, Kd, N, 64, 128) || !map2d(&tx, X, Kd, M, 64, 16)) return ORTHRUS_ERR_ARG;
+  if (!map2d(&tw, W, Kd, N, 64, 128) || !map2d(&tx, X, Kd, M, 64, 16 * (mt_index(M) + 1))) return ORTHRUS_ERR_ARG;
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.partial = (float*)base;

@@ -1,7 +1,7 @@
 // Inline-PTX helpers for sm_100a: mbarriers with bounded waits, TMA tensor
 // loads, and the tcgen05 tensor-core / tensor-memory instructions.
 //
-// Every wait is bounded by wall-clock time (%globaltimer): a wait that runs out
+// Every wait is bounded (SM cycle counter, about 2 s): a wait that runs out
 // records ORTHRUS_ERR_TIMEOUT in the device status word and returns false, so a
 // kernel never spins forever.
 #pragma once
@@ -20,17 +20,21 @@ __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);  // first error wins
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s at 1.965 GHz
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor drains; griddep_wait() blocks
+// until every earlier kernel of the stream has completed and its writes are
+// visible, griddep_launch() lets the next kernel start launching. Both are
+// no-ops for a normal launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // mbarrier
@@ -68,17 +72,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete; false on timeout.
+// The first 4096 polls have no side effects (the common case completes there);
+// after that the wait is bounded by SM cycles (clock64, a register read), about
+// 2 s at the B200's clocks, and then records ORTHRUS_ERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+#pragma unroll 1
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u) {
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        set_status(status, ORTHRUS_ERR_TIMEOUT);
-        return false;
-      }
-      if (status && *(volatile int*)status == ORTHRUS_ERR_TIMEOUT) return false;
+    if ((it & 1023u) == 0u && clock64() - t0 > kWaitLimitCycles) {
+      set_status(status, ORTHRUS_ERR_TIMEOUT);
+      return false;
     }
   }
 }

@@ -27,6 +27,8 @@ struct EmbedArgs {
 //   verify:  ids [y, d_1 .. d_{Q-1}]
 //   prefill: prompt tokens
 __global__ void embed_kernel(const EmbedArgs a) {
+  griddep_wait();
+  griddep_launch();
   const int m = blockIdx.x;
   const int bb = m / a.Q, i = m - bb * a.Q;
   const int b = a.b0 + bb;
@@ -66,6 +68,8 @@ __global__ void embed_kernel(const EmbedArgs a) {
 __global__ void rmsnorm_kernel(const float* __restrict__ h, int D, const float* __restrict__ gain, float eps,
                                __nv_bfloat16* __restrict__ out, int src_first, int src_stride,
                                unsigned long long* reset_keys) {
+  griddep_wait();
+  griddep_launch();
   const int m = blockIdx.x;
   const float* x = h + (size_t)(src_first + m * src_stride) * D;
   __shared__ float red[32];
@@ -98,6 +102,8 @@ __global__ void rmsnorm_kernel(const float* __restrict__ h, int D, const float* 
 
 // token id = lowest index of the row maximum, from the packed 64-bit keys
 __global__ void argmax_finalize_kernel(const unsigned long long* keys, int M, int* dst, int* status) {
+  griddep_wait();
+  griddep_launch();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;
   if (m >= M) return;
   const unsigned long long k = keys[m];
@@ -115,6 +121,8 @@ __global__ void argmax_finalize_kernel(const unsigned long long* keys, int M, in
 //   holds an error (the verify block may not have been written).
 __global__ void accept_kernel(int* pending, const int* draft, const int* ar, int K, int* accept_len, int* committed,
                               int* len, const int* status) {
+  griddep_wait();
+  griddep_launch();
   const int b = blockIdx.x, t = threadIdx.x;
   __shared__ unsigned int masks[3];
   const bool match = t < K && draft[b * K + t] == ar[b * (K + 1) + t];
@@ -148,6 +156,8 @@ __global__ void accept_kernel(int* pending, const int* draft, const int* ar, int
 // with NaN (bf16 0x7FC0), after accept_kernel advanced len.
 __global__ void poison_kernel(__nv_bfloat16* kc, __nv_bfloat16* vc, const int* len, const int* accept_len, int K,
                               int B, int Hkv, int cap, int d) {
+  griddep_wait();
+  griddep_launch();
   const int z = blockIdx.x;  // (l * B + b) * Hkv + h
   const int b = (z / Hkv) % B;
   const int a = accept_len[b];
@@ -162,6 +172,10 @@ __global__ void poison_kernel(__nv_bfloat16* kc, __nv_bfloat16* vc, const int* l
   }
 }
 
-__global__ void set_len_kernel(int* len, int b, int value) { len[b] = value; }
+__global__ void set_len_kernel(int* len, int b, int value) {
+  griddep_wait();
+  griddep_launch();
+  len[b] = value;
+}
 
 }  // namespace orthrus

@@ -19,6 +19,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liborthrus.so")
 
+KIND_NAMES = ["embed", "rmsnorm", "gemm_qkv", "attention", "gemm_o", "gemm_gate_up", "gemm_down", "lm_head",
+              "argmax", "accept", "other", "end"]
+
 OK, ERR_ARG, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_NAN, ERR_UNSUPPORTED, ERR_WORKSPACE = range(8)
 STATUS_NAMES = {0: "OK", 1: "ARG", 2: "CAPACITY", 3: "CUDA", 4: "TIMEOUT", 5: "NAN", 6: "UNSUPPORTED",
                 7: "WORKSPACE"}
@@ -62,6 +65,7 @@ SIGNATURES = [
     ("orthrus_status_ptr", _VP, [_VP]),
     ("orthrus_clear_status", _I32, [_VP, _VP]),
     ("orthrus_decode_step_launches", _I32, [_VP, _I32]),
+    ("orthrus_trace", _I32, [_VP, _VP, _VP, _I32, _VP]),
     ("orthrus_prefill", _I32, [_VP, _VP, _VP, _I32, _VP, _VP]),
     ("orthrus_draft_block", _I32, [_VP, _VP, _I32, _VP, _VP, _VP]),
     ("orthrus_verify_block", _I32, [_VP, _VP, _VP, _I32, _VP, _VP, _VP]),
@@ -248,6 +252,13 @@ class DeviceModel:
 
     def launches_per_step(self, K) -> int:
         return load().orthrus_decode_step_launches(self.plan, K)
+
+    def trace(self, events, kinds, count):
+        """events: ctypes array of cudaEvent_t handles (or None to stop); kinds/count: ctypes int32 arrays."""
+        if events is None:
+            _check("orthrus_trace", load().orthrus_trace(self.plan, None, None, 0, None))
+        else:
+            _check("orthrus_trace", load().orthrus_trace(self.plan, events, kinds, len(events), count))
 
     def read_status(self) -> int:
         return int(self.status.item())
