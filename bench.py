@@ -261,6 +261,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "gemm_down": D * F * 2 + mm * (F * 2 + 2 * D * 4),
         "lm_head": V * D * 2 + mm * D * 2,
         "attention": shape.n_kv_heads * shape.head_dim * 2 * 2 * (n_mean + K) + mm * Hd * 2 * 2,
+        # persistent kernel: one whole forward (draft or verify) per launch, two per step
+        "forward": bytes_total / Ksteps / 2.0,
     }
     for name, b in algo.items():
         if name in kernels:

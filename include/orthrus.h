@@ -157,7 +157,9 @@ enum {
   ORTHRUS_KIND_ARGMAX = 8,     /* argmax finalisation                              */
   ORTHRUS_KIND_ACCEPT = 9,     /* greedy consensus + KV commit                     */
   ORTHRUS_KIND_OTHER = 10,     /* poisoning, length updates, planted-draft copy    */
-  ORTHRUS_KIND_END = 11        /* marker after the last launch of a call          */
+  ORTHRUS_KIND_END = 11,       /* marker after the last launch of a call          */
+  ORTHRUS_KIND_FORWARD = 12    /* persistent kernel: one whole draft or verify forward
+                                  (and, in orthrus_decode_step, the consensus)     */
 };
 
 /* Profiling hook. While set, every launch made by the calls below is preceded

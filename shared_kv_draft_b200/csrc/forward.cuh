@@ -1,0 +1,1173 @@
+// Persistent forward kernel: one launch runs a whole draft-view or verify-view
+// forward of the Orthrus decode step (embedding, every layer's q/k/v
+// projection, block attention, output projection, SwiGLU MLP, final norm, LM
+// head and argmax) for a block of at most 128 token rows, and the verify launch
+// also runs the greedy consensus and KV commit at its end.
+//
+// Why one kernel: at decode sizes every projection is a weight stream of 5-30
+// microseconds, so separate launches pay a start-up and a split-K tail per
+// projection (hundreds per step) that are as long as the stream itself. Here
+// one CTA per SM (cooperative launch, all CTAs co-resident) walks the same list
+// of phases; the phases are ordered by device-wide counters instead of kernel
+// boundaries, and the TMA producer keeps streaming the next phase's weight
+// tiles into its shared-memory ring while the current phase finishes, so the
+// weight stream does not stop at phase boundaries.
+//
+// Phases of one forward (phase p depends on the previous active phase only):
+//   EMBED         h = E[ids], xg = bf16(h * gamma_attn[0]), per-row sums of squares
+//   per layer:
+//     QKV         [xg] W_qkv^T, * rstd, per-head q/k RMSNorm, RoPE; q -> qbuf, K/V ->
+//                 cache slots len+i (verify) or the draft block scratch (draft)
+//     ATTN        block attention over (sequence, kv head, 128-row tile, key chunk) units
+//     COMBINE     merge of the key-chunk partials (only when some slot has several chunks)
+//     O           h += attn W_o^T; xg = bf16(h * gamma_mlp); sums of squares
+//     GU          act = silu(rstd * xg W_g^T) * (rstd * xg W_u^T)
+//     DOWN        h += act W_down^T; xg = bf16(h * gamma_next); sums of squares
+//   LM            logits = rstd * xg W_lm^T; running argmax per row
+// RMSNorm is folded into its neighbours: RMSNorm(h) W^T = diag(rstd) (h*gamma) W^T,
+// so the residual epilogue writes bf16(h * gamma) and 128-column partial sums of
+// h^2, and the consumer multiplies its accumulator rows by rstd, computed from the
+// partial sums in a fixed order (deterministic).
+//
+// Warp roles (224 threads): warp 0 = TMA producer of weight tiles, warp 6 = TMA
+// producer of activation tiles (the loads that wait for the previous phase), warp
+// 1 = tcgen05.mma issuer, warps 2-5 = epilogue (TMEM -> registers -> fused
+// epilogue), attention softmax, embedding and chunk merge. Two issuing threads
+// matter: one thread issuing 8 KB copies streams about 4 TB/s, two reach the
+// HBM rate. Ring stage = a 16 KB "A" slot (a weight tile of 128
+// rows x 64 k, or an attention Q / K / V tile) + an activation slot of Mt x 64.
+#pragma once
+#include "gemm.cuh"
+
+namespace orthrus {
+
+// tensor-map indices: per layer, then global
+// M_WGU3 views W_gate_up as [2][d_ff][d_model] so one box brings 64 gate rows and the
+// 64 matching up rows (one 16 KB TMA copy instead of two 8 KB ones).
+enum { M_WQKV = 0, M_WO, M_WGU, M_WDOWN, M_WDQKV, M_WDO, M_WGU3, M_PER_LAYER };
+// activation maps exist for every token-tile height Mt = 16, 32, ..., 128 (index Mt/16 - 1)
+enum {
+  G_LM = 0,
+  G_Q,
+  G_KC,
+  G_VC,
+  G_KB,
+  G_VB,
+  G_KC64,
+  G_VC64,
+  G_KB64,
+  G_VB64,
+  G_XN,
+  G_ATTN = G_XN + 8,
+  G_ACT = G_ATTN + 8,
+  G_COUNT = G_ACT + 8
+};
+
+enum PhaseKind : int { PH_EMBED = 0, PH_QKV, PH_ATTN, PH_COMBINE, PH_O, PH_GU, PH_DOWN, PH_LM };
+constexpr int kPhasesPerLayer = 6;  // QKV, ATTN, COMBINE, O, GU, DOWN
+constexpr int kFwdThreads = 224;
+constexpr int kMaxStages = 16;
+constexpr int kMaxSlots = 256;        // attention (sequence, kv head, row tile) slots per launch
+constexpr int kMaxChunks = 18;        // key chunks per slot (16 cache chunks + draft block + slack)
+constexpr int kCombineRows = 16;      // rows per merge unit
+constexpr int kScratchBytes = 17408;  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
+
+struct LayerNorms {  // device-resident per-layer gains (fp32)
+  const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
+};
+
+struct FwdArgs {
+  const CUtensorMap* maps;   // device copy: [L][M_PER_LAYER] then [G_COUNT]
+  const LayerNorms* norms;   // device [L]
+  int L, D, H, Hkv, d, F, V, G, qk_norm, mask_id;
+  float eps, scale_log2;
+  double theta;
+  int view;                  // VIEW_DRAFT / VIEW_VERIFY
+  int nb, Q, M, Mt, mt_idx, stages, cap, max_block, batch;
+  int ck;                    // keys per attention chunk: fixed per plan (multiple of 64, >= capacity / 16),
+                             // so a row's softmax runs over the same absolute key chunks whatever
+                             // the block size: verify rows equal the plain AR rows bit for bit
+  const int* pending;        // [nb]
+  const int* draft_ids;      // [nb][Q-1] (verify)
+  int* len;                  // [batch] (read; the fused accept advances it)
+  const __nv_bfloat16* embed;
+  const float* final_norm;
+  __nv_bfloat16 *kc, *vc, *blk_k, *blk_v;
+  float* h;                  // [rows][D]
+  __nv_bfloat16* xg;         // [rows][D]
+  __nv_bfloat16* qbuf;       // [nb][Hkv][Q*G][d]
+  __nv_bfloat16* attn;       // [rows][H*d]
+  __nv_bfloat16* act;        // [rows][F]
+  float2* rope;              // [rows][d/2]
+  float* ss;                 // [D/128][ss_ld] partial sums of squares
+  int ss_ld;
+  unsigned long long* amax;  // [rows]
+  int* out_ids;              // [M] argmax of every row
+  float* logits;             // nullable [M][V]
+  float* partial;            // [2 * grid][128][Mt] split-tile partial sums
+  int* tile_cnt;             // [max tiles] split-tile arrival counters (self-resetting)
+  int* phase_cnt;            // [2 + 6L] completion counters (reset by the last CTA)
+  int* exit_cnt;
+  float* att_o;              // [kMaxSlots][kMaxChunks][128][d]
+  float2* att_ml;            // [kMaxSlots][kMaxChunks][128]
+  int* status;
+  int* diag;                 // [16] where the first timed-out wait gave up (nullable)
+  // greedy consensus fused into the verify launch
+  int accept, K;
+  int* pending_out;          // [nb]
+  int* accept_len;           // [nb]
+  int* committed;            // [nb][K+1]
+};
+
+// Records the first wait that ran out of time: site, phase, ring position and
+// two site-specific values (diag[0] = 1 once written).
+__device__ inline void fwd_diag(const FwdArgs& a, int code, int site, int p, int it, int x0 = 0, int x1 = 0,
+                                int x2 = 0) {
+  if (code != -1 || !a.diag) return;
+  if (atomicCAS(a.diag, 0, 1) != 0) return;
+  a.diag[1] = blockIdx.x;
+  a.diag[2] = threadIdx.x;
+  a.diag[3] = site;
+  a.diag[4] = p;
+  a.diag[5] = it;
+  a.diag[6] = x0;
+  a.diag[7] = x1;
+  a.diag[8] = x2;
+  __threadfence();
+}
+
+__host__ __device__ inline int fwd_n_phases(int L) { return 2 + kPhasesPerLayer * L; }
+__host__ __device__ inline int fwd_phase_kind(int p, int L) {
+  if (p == 0) return PH_EMBED;
+  if (p == 1 + kPhasesPerLayer * L) return PH_LM;
+  return PH_QKV + (p - 1) % kPhasesPerLayer;
+}
+__host__ __device__ inline int fwd_phase_layer(int p) { return (p - 1) / kPhasesPerLayer; }
+
+// Shared memory outside the ring: the attention Q tile (128 rows x d, resident for
+// a whole attention unit, so it cannot live in the ring), the P tile / epilogue
+// staging, small per-CTA tables and the barriers.
+__host__ inline size_t fwd_fixed_smem(int d) {
+  return 1024 /*align*/ + (size_t)128 * d * 2 /*Q*/ + kScratchBytes + 128 * 8 /*red*/ + 128 * 4 /*rstd*/ +
+         128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/;
+}
+__host__ inline size_t fwd_stage_bytes(int Mt) { return 16384 + (size_t)Mt * 128; }
+
+// Shared state every role derives identically at kernel start.
+struct FwdGeom {
+  int rows_per_slot;  // Q * G
+  int rt;             // row tiles per (sequence, kv head)
+  int slots;          // nb * Hkv * rt
+  int CK;             // keys per chunk (multiple of 64)
+  int att_units;      // total attention units
+  int comb_units;     // total merge units (0 when no slot has more than one chunk)
+};
+
+// GEMM phase description
+struct GemmPhase {
+  int epi;            // EPI_QKV / EPI_RESID / EPI_SWIGLU / EPI_ARGMAX
+  int n_tiles, k_chunks;
+  long long units;
+  const CUtensorMap* mw;
+  const CUtensorMap* mx;
+  int gu;             // SwiGLU tile layout (64 gate + 64 up rows)
+};
+
+__device__ inline GemmPhase gemm_phase(const FwdArgs& a, int kind, int l) {
+  GemmPhase g;
+  const CUtensorMap* lm = a.maps + (size_t)l * M_PER_LAYER;
+  const CUtensorMap* gm = a.maps + (size_t)a.L * M_PER_LAYER;
+  const bool draft = a.view == VIEW_DRAFT;
+  g.gu = 0;
+  if (kind == PH_QKV) {
+    g.epi = EPI_QKV;
+    g.n_tiles = (a.H + 2 * a.Hkv) * a.d / 128;
+    g.k_chunks = a.D / 64;
+    g.mw = lm + (draft ? M_WDQKV : M_WQKV);
+    g.mx = gm + G_XN + a.mt_idx;
+  } else if (kind == PH_O) {
+    g.epi = EPI_RESID;
+    g.n_tiles = a.D / 128;
+    g.k_chunks = a.H * a.d / 64;
+    g.mw = lm + (draft ? M_WDO : M_WO);
+    g.mx = gm + G_ATTN + a.mt_idx;
+  } else if (kind == PH_GU) {
+    g.epi = EPI_SWIGLU;
+    g.n_tiles = a.F / 64;
+    g.k_chunks = a.D / 64;
+    g.mw = lm + M_WGU3;
+    g.mx = gm + G_XN + a.mt_idx;
+    g.gu = 1;
+  } else if (kind == PH_DOWN) {
+    g.epi = EPI_RESID;
+    g.n_tiles = a.D / 128;
+    g.k_chunks = a.F / 64;
+    g.mw = lm + M_WDOWN;
+    g.mx = gm + G_ACT + a.mt_idx;
+  } else {  // PH_LM
+    g.epi = EPI_ARGMAX;
+    g.n_tiles = a.V / 128;
+    g.k_chunks = a.D / 64;
+    g.mw = gm + G_LM;
+    g.mx = gm + G_XN + a.mt_idx;
+  }
+  g.units = (long long)g.n_tiles * g.k_chunks;
+  return g;
+}
+
+__device__ inline bool is_gemm_kind(int k) {
+  return k == PH_QKV || k == PH_O || k == PH_GU || k == PH_DOWN || k == PH_LM;
+}
+
+// completion count of a phase
+__device__ inline int phase_target(const FwdArgs& a, const FwdGeom& g, int p) {
+  const int kind = fwd_phase_kind(p, a.L);
+  if (kind == PH_EMBED) return a.M;
+  if (kind == PH_ATTN) return g.att_units;
+  if (kind == PH_COMBINE) return g.comb_units;
+  return gemm_phase(a, kind, 0).n_tiles;
+}
+
+__device__ inline bool phase_active(const FwdGeom& g, int kind) { return kind != PH_COMBINE || g.comb_units > 0; }
+
+// the phase whose completion phase p waits for (the previous active phase)
+__device__ inline int phase_dep(const FwdArgs& a, const FwdGeom& g, int p) {
+  int q = p - 1;
+  if (q >= 1 && !phase_active(g, fwd_phase_kind(q, a.L))) --q;
+  return q;
+}
+
+// ---- attention geometry ------------------------------------------------------
+// slot s = (bb * Hkv + kvh) * rt + r
+__device__ inline int slot_visible_keys(const FwdArgs& a, const FwdGeom& g, const int* lens, int s) {
+  const int r = s % g.rt;
+  const int bb = s / (g.rt * a.Hkv);
+  const int n = min(lens[bb], a.cap);
+  if (a.view == VIEW_DRAFT) return n;  // cache keys; the block is one extra chunk
+  const int row_hi = min(g.rows_per_slot, (r + 1) * 128);
+  const int i_max = (row_hi - 1) / a.G;
+  return min(n + i_max + 1, a.cap);
+}
+
+__device__ inline int slot_chunks(const FwdArgs& a, const FwdGeom& g, const int* lens, int s) {
+  const int vis = slot_visible_keys(a, g, lens, s);
+  const int c = (vis + g.CK - 1) / g.CK;
+  return a.view == VIEW_DRAFT ? c + 1 : max(1, c);
+}
+
+}  // namespace orthrus
+
+namespace orthrus {
+
+struct AttUnit {
+  int slot, chunk, n_chunks, bb, kvh, r, blk, key_lo, key_hi, n, tiles;
+};
+
+// attention unit u -> (slot, key chunk, key range); slot_pre = prefix sums of chunks per slot
+__device__ inline AttUnit att_unit(const FwdArgs& a, const FwdGeom& g, const int* lens, const int* slot_pre, int u) {
+  int lo = 0, hi = g.slots - 1;  // largest s with slot_pre[s] <= u
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (slot_pre[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  AttUnit t;
+  t.slot = lo;
+  t.chunk = u - slot_pre[lo];
+  t.n_chunks = slot_pre[lo + 1] - slot_pre[lo];
+  t.r = lo % g.rt;
+  t.kvh = (lo / g.rt) % a.Hkv;
+  t.bb = lo / (g.rt * a.Hkv);
+  t.n = min(lens[t.bb], a.cap);
+  const int vis = slot_visible_keys(a, g, lens, lo);
+  if (a.view == VIEW_DRAFT && t.chunk == t.n_chunks - 1) {
+    t.blk = 1;
+    t.key_lo = 0;
+    t.key_hi = a.Q;
+  } else {
+    t.blk = 0;
+    t.key_lo = t.chunk * g.CK;
+    t.key_hi = min(vis, t.key_lo + g.CK);
+  }
+  t.tiles = max(1, (t.key_hi - t.key_lo + 63) / 64);
+  return t;
+}
+
+// Residual epilogue of the O and down projections on 32 token rows [m0, m0+32)
+// of one 128-column tile: h += v; xg = bf16(h * gamma_next); partial sum of h^2
+// over the tile's 128 columns per row -> ss[nt][m]. Thread = output column `row`.
+__device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
+                                                   int m_valid, const float* gam, float* epi) {
+  const int D = a.D;
+  const int f = nt * 128 + row;
+  const float gf = gam[f];
+  float hv[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) hv[j] = (m0 + j < m_valid) ? __ldcg(a.h + (size_t)(m0 + j) * D + f) : 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (m0 + j < m_valid) {
+      hv[j] += v[j];
+      a.h[(size_t)(m0 + j) * D + f] = hv[j];
+      a.xg[(size_t)(m0 + j) * D + f] = __float2bfloat16(hv[j] * gf);
+    }
+    epi[j * kEpiStride + row] = hv[j] * hv[j];
+  }
+  named_bar_sync(1, 128);
+  {
+    const int t = threadIdx.x - 64;
+    const int j = t >> 2, q = t & 3;
+    float s = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) s += epi[j * kEpiStride + q * 32 + i];
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (q == 0 && m0 + j < m_valid) a.ss[(size_t)nt * a.ss_ld + m0 + j] = s;
+  }
+  named_bar_sync(1, 128);
+}
+
+// Epilogue of one 32-row group for the GEMM phase kinds. Consumers of a
+// normalised input first scale by rstd of the token row.
+__device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const GemmArgs& ga, int epi_kind, float* v, int row,
+                                             int m0, int nt, int m_valid, float* epi, unsigned long long* red,
+                                             const float* rstd_s, const float* gam) {
+  if (epi_kind == EPI_RESID) {
+    fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam, epi);
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] *= rstd_s[m0 + j];
+  if (epi_kind == EPI_QKV) epilogue_group<EPI_QKV>(ga, v, row, m0, 0, nt, m_valid, epi, red);
+  else if (epi_kind == EPI_SWIGLU) epilogue_group<EPI_SWIGLU>(ga, v, row, m0, 0, nt, m_valid, epi, red);
+  else epilogue_group<EPI_ARGMAX>(ga, v, row, m0, 0, nt, m_valid, epi, red);
+}
+
+}  // namespace orthrus
+
+namespace orthrus {
+
+// Greedy consensus (verify launch) and counter reset; run by the last CTA to
+// finish, when every other CTA has left the kernel.
+__device__ inline void fwd_finalize(const FwdArgs& a, int n_ph) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  for (int m = t; m < a.M; m += blockDim.x) {
+    const unsigned long long k = __ldcg(a.amax + m);
+    int id = 0;
+    if (k == 0ull) set_status(a.status, ORTHRUS_ERR_NAN);
+    else id = (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    a.out_ids[m] = id;
+  }
+  __syncthreads();
+  if (a.accept) {
+    const bool err = *(volatile int*)a.status != 0;
+    const int K = a.K;
+    for (int b = warp; b < a.nb; b += blockDim.x >> 5) {
+      // accept length = index of the first draft that differs from the AR argmax before it
+      int acc = K;
+      for (int i0 = 0; i0 < K; i0 += 32) {
+        const int i = i0 + lane;
+        const bool mism = i < K && a.draft_ids[b * K + i] != a.out_ids[b * (K + 1) + i];
+        const unsigned bal = __ballot_sync(0xffffffffu, mism);
+        if (bal) {
+          acc = i0 + __ffs(bal) - 1;
+          break;
+        }
+      }
+      for (int i = lane; i <= K; i += 32) {
+        int v = -1;
+        if (!err && i < acc) v = a.draft_ids[b * K + i];
+        else if (!err && i == acc) v = a.out_ids[b * (K + 1) + acc];
+        a.committed[b * (K + 1) + i] = v;
+      }
+      if (lane == 0) {
+        if (err) {
+          a.accept_len[b] = -1;
+        } else {
+          a.accept_len[b] = acc;
+          a.pending_out[b] = a.out_ids[b * (K + 1) + acc];
+          a.len[b] += acc + 1;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = t; i < n_ph; i += blockDim.x) a.phase_cnt[i] = 0;
+  if (t == 0) *a.exit_cnt = 0;
+  __threadfence();
+}
+
+// Epilogue warps (2-5) of the persistent forward kernel.
+template <int D_HEAD>
+__device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeom& g, uint8_t* smem,
+                                                  uint32_t stage_bytes, int S, uint8_t* scr,
+                                                  unsigned long long* red, float* rstd_s, const int* lens_s,
+                                                  const int* slot_pre, uint64_t* accf, uint64_t* acce,
+                                                  uint64_t* full, uint64_t* s_full, uint64_t* p_full,
+                                                  uint64_t* o_full, uint64_t* t_done, int* flag,
+                                                  uint32_t tmem_base, uint32_t tS, uint32_t tO) {
+  constexpr int d = D_HEAD;
+  constexpr int halves = d / 64;
+  float* epi = (float*)scr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int et = threadIdx.x - 64;  // 0..127
+  const int ew = warp - 2;          // 0..3
+  const int quarter = warp & 3;     // TMEM lane quarter this warp may access
+  const int row = quarter * 32 + lane;
+  const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+  const int Gd = gridDim.x, c = blockIdx.x;
+  const int n_ph = fwd_n_phases(a.L);
+  const int D = a.D;
+  int seg = 0, ta = 0, it = 0, acq = -1, bc = 0;
+  bool ok = true;
+
+  // one thread waits, the result is shared by the four warps (rotating flag slots
+  // keep a slow reader from seeing the next call's value)
+  auto bcast = [&](bool v_from_thread0) -> bool {
+    const int slot = 1 + (bc++ & 3);
+    if (et == 0) flag[slot] = v_from_thread0 ? 1 : 0;
+    named_bar_sync(1, 128);
+    return flag[slot] != 0;
+  };
+  int cur_p = 0;
+  auto acquire_phase = [&](int dep) -> bool {
+    if (dep <= acq) return true;
+    bool r = false;
+    if (et == 0) {
+      const int tgt = phase_target(a, g, dep);
+      const int code = wait_count_code(a.phase_cnt + dep, tgt, a.status);
+      fwd_diag(a, code, 12, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
+      r = code == 1;
+    }
+    r = bcast(r);
+    if (r) {
+      (void)ld_acquire_gpu(a.phase_cnt + dep);
+      acq = dep;
+    }
+    return r;
+  };
+  auto signal = [&](int p) {
+    fence_proxy_async_global();
+    __threadfence();
+    named_bar_sync(1, 128);
+    if (et == 0) red_release_gpu_add(a.phase_cnt + p, 1);
+  };
+  auto bar_wait_all = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+    bool r = false;
+    if (et == 0) {
+      const int code = mbar_wait_code(bar, parity, a.status);
+      fwd_diag(a, code, site, cur_p, it, (int)parity, ta, seg);
+      r = code == 1;
+    }
+    return bcast(r);
+  };
+
+  for (int p = 0; ok && p < n_ph; ++p) {
+    const int kind = fwd_phase_kind(p, a.L);
+    if (!phase_active(g, kind)) continue;
+    const int l = fwd_phase_layer(p);
+    const int dep = phase_dep(a, g, p);
+    cur_p = p;
+
+    if (kind == PH_EMBED) {
+      // ---------------- embedding rows ----------------
+      const float* g0 = a.norms[0].attn_norm;
+      const int parts = D / 128;
+      for (int m = c; m < a.M; m += Gd) {
+        const int bb = m / a.Q, i = m - bb * a.Q;
+        int id;
+        if (i == 0) id = a.pending[bb];
+        else id = a.view == VIEW_DRAFT ? a.mask_id : a.draft_ids[bb * (a.Q - 1) + i - 1];
+        if (id < 0 || id >= a.V) {
+          if (et == 0) set_status(a.status, ORTHRUS_ERR_ARG);
+          id = 0;
+        }
+        const int n = lens_s[bb];
+        if (et == 0 && i == 0 && a.view == VIEW_VERIFY && n + a.Q > a.cap) set_status(a.status, ORTHRUS_ERR_CAPACITY);
+        const __nv_bfloat16* src = a.embed + (size_t)id * D;
+        for (int pp = 0; pp < parts; ++pp) {
+          const int col = pp * 128 + et;
+          const float x = __bfloat162float(src[col]);
+          a.h[(size_t)m * D + col] = x;
+          a.xg[(size_t)m * D + col] = __float2bfloat16(x * g0[col]);
+          const float s = warp_sum(x * x);
+          if (lane == 0) epi[ew * 64 + pp] = s;
+        }
+        named_bar_sync(1, 128);
+        if (et < parts) a.ss[(size_t)et * a.ss_ld + m] = ((epi[et] + epi[64 + et]) + epi[128 + et]) + epi[192 + et];
+        if (et < d / 2) {
+          const double ang = (double)(n + i) * pow(a.theta, -2.0 * (double)et / (double)d);
+          a.rope[(size_t)m * (d / 2) + et] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+        if (et == 0) a.amax[m] = 0ull;
+        named_bar_sync(1, 128);
+        signal(p);
+      }
+    } else if (is_gemm_kind(kind)) {
+      // ---------------- projection epilogues ----------------
+      const GemmPhase gp = gemm_phase(a, kind, l);
+      const long long W = gp.units;
+      const long long u0 = unit_start(W, Gd, c), u1 = unit_start(W, Gd, c + 1);
+      const int kc = gp.k_chunks;
+      if (u0 == u1) continue;
+      if (!acquire_phase(dep)) {
+        ok = false;
+        break;
+      }
+      if (kind == PH_QKV || kind == PH_GU || kind == PH_LM) {
+        if (et < a.Mt) {
+          float s = 0.f;
+          if (et < a.M)
+            for (int pp = 0; pp < D / 128; ++pp) s += __ldcg(a.ss + (size_t)pp * a.ss_ld + et);
+          rstd_s[et] = et < a.M ? rsqrtf(s / (float)D + a.eps) : 0.f;
+        }
+        named_bar_sync(1, 128);
+      }
+      GemmArgs ga;
+      memset(&ga, 0, sizeof(ga));
+      ga.M = a.M;
+      ga.Mt = a.Mt;
+      ga.status = a.status;
+      ga.out_bf16 = a.act;
+      ga.ld_out = a.F;
+      ga.amax = a.amax;
+      ga.logits = a.logits;
+      ga.ld_logits = a.V;
+      const float* gam = nullptr;
+      if (kind == PH_QKV) {
+        const bool dv = a.view == VIEW_DRAFT;
+        QkvEpi& q = ga.qkv;
+        q.H = a.H;
+        q.Hkv = a.Hkv;
+        q.d = d;
+        q.Q = a.Q;
+        q.b0 = 0;
+        q.qk_norm = a.qk_norm;
+        q.mode = a.view;
+        q.eps = a.eps;
+        q.gq = dv ? a.norms[l].wd_q_norm : a.norms[l].q_norm;
+        q.gk = dv ? a.norms[l].wd_k_norm : a.norms[l].k_norm;
+        q.rope = a.rope;
+        q.len = a.len;
+        q.qbuf = a.qbuf;
+        if (dv) {
+          const size_t lo = (size_t)l * a.batch * a.Hkv * a.max_block * d;
+          q.kdst = a.blk_k + lo;
+          q.vdst = a.blk_v + lo;
+          q.kv_stride = a.max_block;
+        } else {
+          const size_t lo = (size_t)l * a.batch * a.Hkv * a.cap * d;
+          q.kdst = a.kc + lo;
+          q.vdst = a.vc + lo;
+          q.kv_stride = a.cap;
+        }
+      } else if (kind == PH_O) {
+        gam = a.norms[l].mlp_norm;
+      } else if (kind == PH_DOWN) {
+        gam = l + 1 < a.L ? a.norms[l + 1].attn_norm : a.final_norm;
+      }
+      const int first_tile = (int)(u0 / kc);
+      long long u = u0;
+      while (ok && u < u1) {
+        const int t = (int)(u / kc);
+        const long long seg_start = u, seg_end = min(u1, (long long)(t + 1) * kc);
+        u = seg_end;
+        const int buf = seg & 1, use = seg >> 1;
+        ++seg;
+        if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nt = t;
+        const int m_valid = min(a.Mt, a.M);
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * 128;
+        const bool whole = seg_start == (long long)t * kc && seg_end == (long long)(t + 1) * kc;
+        float v[32];
+        if (whole) {
+          for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+            tmem_ld32(taddr + m0, v);
+            fwd_epilogue(a, ga, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce[buf]);
+          signal(p);
+        } else {
+          const int slot = 2 * c + (t == first_tile ? 0 : 1);
+          float* part = a.partial + (size_t)slot * (128 * 128) + (size_t)row * a.Mt;
+          for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+            tmem_ld32(taddr + m0, v);
+            const int n4 = min(32, a.Mt - m0) / 4;
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq)
+              if (qq < n4)
+                __stcg(reinterpret_cast<float4*>(part + m0) + qq,
+                       make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce[buf]);
+          // contributors: the CTAs with a non-empty unit range inside the tile (with
+          // fewer units than CTAs, CTAs between two owners may have none)
+          const int c_lo = unit_owner((long long)t * kc, W, Gd);
+          const int c_hi = unit_owner((long long)(t + 1) * kc - 1, W, Gd);
+          int n_contrib = 0;
+          for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += unit_start(W, Gd, cc + 1) > unit_start(W, Gd, cc);
+          __threadfence();
+          named_bar_sync(1, 128);
+          bool last = false;
+          if (et == 0) last = atomicAdd(a.tile_cnt + t, 1) == n_contrib - 1;
+          last = bcast(last);
+          if (last) {
+            __threadfence();
+            if (et == 0) a.tile_cnt[t] = 0;
+            for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+              const int n4 = min(32, a.Mt - m0) / 4;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = 0.f;
+              for (int cc = c_lo; cc <= c_hi; ++cc) {  // fixed k order
+                if (unit_start(W, Gd, cc + 1) == unit_start(W, Gd, cc)) continue;  // no units, no partial
+                const int ft = (int)(unit_start(W, Gd, cc) / kc);
+                const float4* pp = reinterpret_cast<const float4*>(
+                    a.partial + (size_t)(2 * cc + (t == ft ? 0 : 1)) * (128 * 128) + (size_t)row * a.Mt + m0);
+                float4 x[8];
+#pragma unroll
+                for (int qq = 0; qq < 8; ++qq) x[qq] = qq < n4 ? __ldcg(pp + qq) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int qq = 0; qq < 8; ++qq) {
+                  v[4 * qq] += x[qq].x;
+                  v[4 * qq + 1] += x[qq].y;
+                  v[4 * qq + 2] += x[qq].z;
+                  v[4 * qq + 3] += x[qq].w;
+                }
+              }
+              fwd_epilogue(a, ga, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
+            }
+            signal(p);
+          }
+        }
+      }
+      it += (int)(u1 - u0);
+    } else if (kind == PH_ATTN) {
+      // ---------------- block attention (thread = query row of the tile) ----------------
+      if (c >= g.att_units) continue;
+      if (!acquire_phase(dep)) {
+        ok = false;
+        break;
+      }
+      for (int u = c; ok && u < g.att_units; u += Gd) {
+        const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
+        const int grow = t.r * 128 + row;
+        const bool row_ok = grow < g.rows_per_slot;
+        const int i = row_ok ? grow / a.G : 0;
+        const int row_hi = min(g.rows_per_slot, (t.r + 1) * 128);
+        const int i_max = (row_hi - 1) / a.G;
+        int lim = t.key_hi, kv_end = t.key_hi;
+        if (a.view == VIEW_VERIFY) {
+          lim = min(t.n + i + 1, t.key_hi);
+          kv_end = min(t.n + i_max + 1, t.key_hi);
+        }
+        if (!row_ok) lim = t.key_lo;
+        float o[d];
+#pragma unroll
+        for (int e = 0; e < d; ++e) o[e] = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;
+        for (int j = 0; j < t.tiles; ++j, it += 2, ++ta) {
+          if (!bar_wait_all(s_full, (uint32_t)ta & 1u, 14)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int key0 = t.key_lo + j * 64;
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            float v[32];
+            tmem_ld32(tS + lane_base + c0, v);
+#pragma unroll
+            for (int tt = 0; tt < 32; ++tt)
+              if (key0 + c0 + tt < lim) mx = fmaxf(mx, v[tt] * a.scale_log2);
+          }
+          const float m_new = fmaxf(m_run, mx);
+          const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+          float sum = 0.f;
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            float v[32];
+            tmem_ld32(tS + lane_base + c0, v);
+            uint32_t pk[16];
+#pragma unroll
+            for (int tt = 0; tt < 32; tt += 2) {
+              const float p0 = (key0 + c0 + tt < lim) ? exp2f(v[tt] * a.scale_log2 - m_new) : 0.f;
+              const float p1 = (key0 + c0 + tt + 1 < lim) ? exp2f(v[tt + 1] * a.scale_log2 - m_new) : 0.f;
+              sum += p0 + p1;
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              pk[tt / 2] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            uint8_t* rowp = scr + row * 128;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int ch = (c0 >> 3) + q4;
+              *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) =
+                  make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            }
+          }
+          l_run = l_run * alpha + sum;
+          // V rows of keys no row may see are zeroed (stale or poisoned cache rows)
+          if (key0 + 64 > kv_end && row < 64 && key0 + row >= kv_end) {
+            const int vs = (it + 1) % S;
+            if (mbar_wait_abortable(&full[vs], (uint32_t)((it + 1) / S) & 1u, a.status)) {
+              uint8_t* vb = smem + (size_t)vs * stage_bytes;
+#pragma unroll
+              for (int hh = 0; hh < halves; ++hh) {
+                uint4* vr = reinterpret_cast<uint4*>(vb + hh * 8192 + row * 128);
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) vr[q8] = make_uint4(0u, 0u, 0u, 0u);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full);
+          if (!bar_wait_all(o_full, (uint32_t)ta & 1u, 15)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < d; c0 += 32) {
+            float v[32];
+            tmem_ld32(tO + lane_base + c0, v);
+#pragma unroll
+            for (int tt = 0; tt < 32; ++tt) o[c0 + tt] = o[c0 + tt] * alpha + v[tt];
+          }
+          m_run = m_new;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(t_done);
+        }
+        if (!ok) break;
+        const int H = a.H;
+        if (t.n_chunks == 1) {
+          if (row_ok) {
+            const int gg = grow - i * a.G;
+            __nv_bfloat16* dst = a.attn + ((size_t)(t.bb * a.Q + i) * H + t.kvh * a.G + gg) * d;
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+            for (int e = 0; e < d; e += 8) {
+              __nv_bfloat162 hb[4];
+#pragma unroll
+              for (int tt = 0; tt < 4; ++tt) hb[tt] = __floats2bfloat162_rn(o[e + 2 * tt] * inv, o[e + 2 * tt + 1] * inv);
+              *reinterpret_cast<uint4*>(dst + e) = *reinterpret_cast<uint4*>(hb);
+            }
+          }
+        } else {
+          const size_t pidx = ((size_t)t.slot * kMaxChunks + t.chunk) * 128 + row;
+          float* po = a.att_o + pidx * d;
+#pragma unroll
+          for (int e = 0; e < d; e += 4) __stcg(reinterpret_cast<float4*>(po + e), make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
+          __stcg(a.att_ml + pidx, make_float2(m_run, l_run));
+        }
+        signal(p);
+      }
+    } else if (kind == PH_COMBINE) {
+      // ---------------- merge of key-chunk partials ----------------
+      if (c >= g.comb_units) continue;
+      if (!acquire_phase(dep)) {
+        ok = false;
+        break;
+      }
+      constexpr int per = d / 8;  // columns per thread
+      for (int u = c; u < g.comb_units; u += Gd) {
+        const int slot = u / (128 / kCombineRows), grp = u % (128 / kCombineRows);
+        const int nch = slot_pre[slot + 1] - slot_pre[slot];
+        const int r_t = slot % g.rt, kvh = (slot / g.rt) % a.Hkv, bb = slot / (g.rt * a.Hkv);
+        const int r = grp * kCombineRows + (et >> 3), sub = et & 7;
+        const int grow = r_t * 128 + r;
+        if (nch > 1 && grow < g.rows_per_slot) {
+          const int i = grow / a.G, gg = grow - i * a.G;
+          const float2* ml = a.att_ml + (size_t)slot * kMaxChunks * 128 + r;
+          float mstar = -INFINITY;
+          for (int ch = 0; ch < nch; ++ch) mstar = fmaxf(mstar, __ldcg(ml + ch * 128).x);
+          float L = 0.f;
+          float acc[per];
+#pragma unroll
+          for (int e = 0; e < per; ++e) acc[e] = 0.f;
+          for (int ch = 0; ch < nch; ++ch) {
+            const float2 v = __ldcg(ml + ch * 128);
+            const float w = (v.x == -INFINITY) ? 0.f : exp2f(v.x - mstar);
+            L += v.y * w;
+            const float4* po = reinterpret_cast<const float4*>(
+                a.att_o + (((size_t)slot * kMaxChunks + ch) * 128 + r) * d + sub * per);
+#pragma unroll
+            for (int e = 0; e < per / 4; ++e) {
+              const float4 x = __ldcg(po + e);
+              acc[4 * e] += w * x.x;
+              acc[4 * e + 1] += w * x.y;
+              acc[4 * e + 2] += w * x.z;
+              acc[4 * e + 3] += w * x.w;
+            }
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          __nv_bfloat16* dst = a.attn + ((size_t)(bb * a.Q + i) * a.H + kvh * a.G + gg) * d + sub * per;
+#pragma unroll
+          for (int e = 0; e < per; e += 8) {
+            __nv_bfloat162 hb[4];
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) hb[tt] = __floats2bfloat162_rn(acc[e + 2 * tt] * inv, acc[e + 2 * tt + 1] * inv);
+            *reinterpret_cast<uint4*>(dst + e) = *reinterpret_cast<uint4*>(hb);
+          }
+        }
+        signal(p);
+      }
+    }
+  }
+}
+
+}  // namespace orthrus
+
+namespace orthrus {
+
+template <int D_HEAD>
+__global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_constant__ FwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  constexpr int d = D_HEAD;
+  constexpr int halves = d / 64;
+  const int S = a.stages;
+  const uint32_t x_bytes = (uint32_t)a.Mt * 128u;
+  const uint32_t stage_bytes = 16384u + x_bytes;
+  uint8_t* sQ = smem + (size_t)S * stage_bytes;   // attention Q tile, d/64 blocks of 128 rows x 64
+  uint8_t* scr = sQ + (size_t)128 * d * 2;         // P tile / epilogue staging
+  unsigned long long* red = (unsigned long long*)(scr + kScratchBytes);
+  float* rstd_s = (float*)(red + 128);
+  int* lens_s = (int*)(rstd_s + 128);
+  int* slot_pre = lens_s + 128;
+  uint64_t* bars = (uint64_t*)(((uintptr_t)(slot_pre + kMaxSlots + 1) + 7) & ~(uintptr_t)7);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kMaxStages;
+  uint64_t* accf = bars + 2 * kMaxStages;  // [2]
+  uint64_t* acce = accf + 2;               // [2]
+  uint64_t* s_full = acce + 2;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_full = s_full + 2;
+  uint64_t* t_done = s_full + 3;
+  uint64_t* done = s_full + 4;
+  uint64_t* q_full = s_full + 5;
+  uint64_t* q_empty = s_full + 6;
+  uint32_t* tmem_slot = (uint32_t*)(q_empty + 1);
+  int* flag = (int*)(tmem_slot + 1);  // [8]
+  FwdGeom* geom_s = (FwdGeom*)(flag + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Gd = gridDim.x, c = blockIdx.x;
+  const int n_ph = fwd_n_phases(a.L);
+  auto stage_ptr = [&](int s) { return smem + (size_t)s * stage_bytes; };
+
+  // ---------------- set-up ----------------
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 2);  // one arrival from each producer
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 4);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(o_full, 1);
+    mbar_init(t_done, 4);
+    mbar_init(done, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    fence_barrier_init();
+  }
+  if (threadIdx.x < a.nb) lens_s[threadIdx.x] = a.len[threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    FwdGeom g;
+    g.rows_per_slot = a.Q * a.G;
+    g.rt = (g.rows_per_slot + 127) / 128;
+    g.slots = a.nb * a.Hkv * g.rt;
+    g.CK = a.ck;
+    slot_pre[0] = 0;
+    bool multi = false;
+    for (int s = 0; s < g.slots; ++s) {
+      const int ch = slot_chunks(a, g, lens_s, s);
+      multi = multi || ch > 1;
+      slot_pre[s + 1] = slot_pre[s] + ch;
+    }
+    g.att_units = slot_pre[g.slots];
+    g.comb_units = multi ? g.slots * (128 / kCombineRows) : 0;
+    *geom_s = g;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const FwdGeom g = *geom_s;
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tS = tmem_base + 256;  // attention scores: 64 columns
+  const uint32_t tO = tmem_base + 320;  // attention P V tile: d columns
+
+  if (warp == 0 || warp == 6) {
+    // ============ TMA producers: warp 0 streams weight tiles, warp 6 activations ============
+    // Both walk the same ring; a stage's full barrier expects one arrival from each.
+    // The weight producer never waits for a dependency, so it runs up to a ring ahead
+    // into the next phase while the activation producer waits for the phase before.
+    if (lane == 0) {
+      const bool wprod = warp == 0;
+      const CUtensorMap* gm = a.maps + (size_t)a.L * M_PER_LAYER;
+      const uint64_t pol_w = policy_evict_first();
+      int last_ph[kMaxStages];
+      for (int s = 0; s < kMaxStages; ++s) last_ph[s] = -1;
+      int known_done = -1;
+      bool ok = true;
+      int it = 0, qu = 0;
+      int cur_p = 0;
+      auto dep_ready = [&](int dep) -> bool {
+        if (dep <= known_done) return true;
+        const int tgt = phase_target(a, g, dep);
+        const int r = wait_count_code(a.phase_cnt + dep, tgt, a.status);
+        if (r != 1) {
+          fwd_diag(a, r, 3, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
+          return false;
+        }
+        known_done = dep;
+        fence_proxy_async_global();
+        return true;
+      };
+      for (int p = 0; ok && p < n_ph; ++p) {
+        const int kind = fwd_phase_kind(p, a.L);
+        if (!phase_active(g, kind)) continue;
+        const int l = fwd_phase_layer(p);
+        const int dep = phase_dep(a, g, p);
+        cur_p = p;
+        if (is_gemm_kind(kind)) {
+          const GemmPhase gp = gemm_phase(a, kind, l);
+          const long long W = gp.units;
+          const long long u0 = unit_start(W, Gd, c), u1 = unit_start(W, Gd, c + 1);
+          const int kc = gp.k_chunks;
+          for (long long u = u0; u < u1; ++u, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (uint32_t)(it / S) & 1u;
+            const int r = mbar_wait_code(&empty[s], ph ^ 1u, a.status);
+            if (r != 1) {
+              fwd_diag(a, r, wprod ? 1 : 2, p, it, s);
+              ok = false;
+              break;
+            }
+            const int t = (int)(u / kc), k = (int)(u - (long long)t * kc);
+            uint8_t* st = stage_ptr(s);
+            if (wprod) {
+              mbar_arrive_expect_tx(&full[s], 16384u);
+              if (gp.gu) tma_load_3d_hint(st, gp.mw, &full[s], k * 64, t * 64, 0, pol_w);  // 64 gate + 64 up rows
+              else tma_load_2d_hint(st, gp.mw, &full[s], k * 64, t * 128, pol_w);
+            } else {
+              if (!dep_ready(dep)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(&full[s], x_bytes);
+              tma_load_2d(st + 16384, gp.mx, &full[s], k * 64, 0);
+            }
+            last_ph[s] = (int)ph;
+          }
+        } else if (kind == PH_ATTN) {
+          for (int u = c; ok && u < g.att_units; u += Gd, ++qu) {
+            const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
+            const int zc = (l * a.batch + t.bb) * a.Hkv + t.kvh;
+            const int qrow = (t.bb * a.Hkv + t.kvh) * g.rows_per_slot + t.r * 128;
+            const int n_loads = 2 * t.tiles;
+            if (!wprod) {  // Q tile into its own region once the previous unit's S MMAs are done
+              const int r = mbar_wait_code(q_empty, ((uint32_t)qu & 1u) ^ 1u, a.status);
+              if (r != 1) fwd_diag(a, r, 4, p, it, qu);
+              if (r != 1 || !dep_ready(dep)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(q_full, 16384u * halves);
+              for (int hh = 0; hh < halves; ++hh) tma_load_2d(sQ + hh * 16384, gm + G_Q, q_full, hh * 64, qrow);
+            }
+            for (int j = 0; j < n_loads; ++j, ++it) {
+              const int s = it % S;
+              const uint32_t ph = (uint32_t)(it / S) & 1u;
+              const int r = mbar_wait_code(&empty[s], ph ^ 1u, a.status);
+              if (r != 1) {
+                fwd_diag(a, r, wprod ? 1 : 2, p, it, s, 1);
+                ok = false;
+                break;
+              }
+              last_ph[s] = (int)ph;
+              if (wprod) {
+                mbar_arrive(&full[s]);  // attention tiles all come from the activation producer
+                continue;
+              }
+              if (!dep_ready(dep)) {
+                ok = false;
+                break;
+              }
+              uint8_t* st = stage_ptr(s);
+              const int key0 = t.key_lo + (j >> 1) * 64;
+              const bool is_v = j & 1;
+              const CUtensorMap* mp = t.blk ? (is_v ? gm + G_VB64 : gm + G_KB64) : (is_v ? gm + G_VC64 : gm + G_KC64);
+              mbar_arrive_expect_tx(&full[s], 8192u * halves);
+              for (int hh = 0; hh < halves; ++hh) tma_load_3d(st + hh * 8192, mp, &full[s], hh * 64, key0, zc);
+            }
+          }
+        }
+      }
+      if (ok) {
+        for (int s = 0; s < S; ++s)
+          if (last_ph[s] >= 0) fwd_diag(a, mbar_wait_code(&full[s], (uint32_t)last_ph[s], a.status), 16, n_ph, it, s);
+      }
+      if (!ok || *(volatile int*)a.status != 0) {
+        sleep_ns(20000);  // let loads already in flight land before the CTA can exit
+        sleep_ns(20000);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      const uint32_t idesc_g = idesc_bf16(128, a.Mt, false);
+      const uint32_t idS = idesc_bf16(128, 64, false);
+      const uint32_t idO = idesc_bf16(128, d, true);
+      const uint32_t pa = smem_u32(scr);
+      int it = 0, seg = 0, ta = 0, qu = 0;
+      bool ok = true;
+      for (int p = 0; ok && p < n_ph; ++p) {
+        const int kind = fwd_phase_kind(p, a.L);
+        if (!phase_active(g, kind)) continue;
+        const int l = fwd_phase_layer(p);
+        if (is_gemm_kind(kind)) {
+          const GemmPhase gp = gemm_phase(a, kind, l);
+          const long long W = gp.units;
+          const long long u0 = unit_start(W, Gd, c), u1 = unit_start(W, Gd, c + 1);
+          const int kc = gp.k_chunks;
+          long long u = u0;
+          while (ok && u < u1) {
+            const int t = (int)(u / kc);
+            const long long seg_start = u, seg_end = min(u1, (long long)(t + 1) * kc);
+            const int buf = seg & 1, use = seg >> 1;
+            int r = mbar_wait_code(&acce[buf], (uint32_t)(use & 1) ^ 1u, a.status);
+            if (r != 1) {
+              fwd_diag(a, r, 5, p, it, seg);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + buf * 128;
+            for (; u < seg_end; ++u, ++it) {
+              const int s = it % S;
+              const uint32_t ph = (uint32_t)(it / S) & 1u;
+              r = mbar_wait_code(&full[s], ph, a.status);
+              if (r != 1) {
+                fwd_diag(a, r, 6, p, it, s);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t wa = smem_u32(stage_ptr(s));
+              const uint32_t xa = wa + 16384;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(d_tmem, sw128_desc(wa + kk * 32, 16, 1024), sw128_desc(xa + kk * 32, 16, 1024), idesc_g,
+                            (u > seg_start || kk > 0) ? 1u : 0u);
+              mma_commit(&empty[s]);
+            }
+            if (!ok) break;
+            mma_commit(&accf[buf]);
+            ++seg;
+          }
+        } else if (kind == PH_ATTN) {
+          const uint32_t qa = smem_u32(sQ);
+          for (int u = c; ok && u < g.att_units; u += Gd, ++qu) {
+            const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
+            int r = mbar_wait_code(q_full, (uint32_t)qu & 1u, a.status);
+            if (r != 1) {
+              fwd_diag(a, r, 7, p, it, qu);
+              ok = false;
+              break;
+            }
+            for (int j = 0; ok && j < t.tiles; ++j, it += 2, ++ta) {
+              const int ks = it % S, vs = (it + 1) % S;
+              r = mbar_wait_code(&full[ks], (uint32_t)(it / S) & 1u, a.status);
+              if (r != 1) {
+                fwd_diag(a, r, 8, p, it, ks);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t ka = smem_u32(stage_ptr(ks));
+#pragma unroll
+              for (int kk = 0; kk < d / 16; ++kk)
+                mma_bf16_ss(tS, sw128_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                            sw128_desc(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+              mma_commit(s_full);
+              mma_commit(&empty[ks]);
+              if (j == t.tiles - 1) mma_commit(q_empty);  // last read of this unit's Q tile
+              r = mbar_wait_code(p_full, (uint32_t)ta & 1u, a.status);
+              if (r == 1) {
+                r = mbar_wait_code(&full[vs], (uint32_t)((it + 1) / S) & 1u, a.status);
+                if (r == 1 && ta > 0) {
+                  r = mbar_wait_code(t_done, (uint32_t)(ta - 1) & 1u, a.status);
+                  if (r != 1) fwd_diag(a, r, 11, p, it, ta);
+                } else if (r != 1) {
+                  fwd_diag(a, r, 10, p, it, vs);
+                }
+              } else {
+                fwd_diag(a, r, 9, p, it, ta);
+              }
+              if (r != 1) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t va = smem_u32(stage_ptr(vs));
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, 8192, 1024), idO,
+                            kk > 0 ? 1u : 0u);
+              mma_commit(o_full);
+              mma_commit(&empty[vs]);
+            }
+            if (!ok) break;
+          }
+        }
+      }
+      mma_commit(done);
+      mbar_wait(done, 0, a.status);
+    }
+  } else {
+    // ======================= epilogue warps =======================
+    fwd_epilogue_role<D_HEAD>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, accf, acce, full,
+                              s_full, p_full, o_full, t_done, flag, tmem_base, tS, tO);
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int old = atomicAdd(a.exit_cnt, 1);
+    flag[7] = (old == Gd - 1) ? 1 : 0;
+  }
+  __syncthreads();
+  if (flag[7]) {
+    __threadfence();
+    fwd_finalize(a, n_ph);
+  }
+}
+
+}  // namespace orthrus

@@ -11,6 +11,7 @@
 #include <utility>
 
 #include "attention.cuh"
+#include "forward.cuh"
 #include "gemm.cuh"
 #include "orthrus.h"
 #include "small.cuh"
@@ -51,13 +52,14 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint3
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D bf16 map over [z][rows][cols]; box = 64 cols x 128 rows x 1.
-bool map3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t z) {
+// 3D bf16 map over [z][rows][cols]; box = 64 cols x box_rows rows x box_z.
+bool map3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t z, uint32_t box_rows = 128,
+           uint32_t box_z = 1) {
   EncodeTiledFn f = encode_fn();
   if (!f || !base) return false;
   cuuint64_t dims[3] = {cols, rows, z};
   cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, box_z};
   cuuint32_t es[3] = {1, 1, 1};
   return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -116,9 +118,6 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // plan
 // ---------------------------------------------------------------------------
 constexpr uint64_t kPlanMagic = 0x4F52544852555331ull;  // "ORTHRUS1"
-enum { M_WQKV = 0, M_WO, M_WGU, M_WDOWN, M_WDQKV, M_WDO, M_PER_LAYER };
-// activation maps exist for every token-tile height Mt = 16, 32, ..., 128 (index Mt/16 - 1)
-enum { G_LM = 0, G_Q, G_KC, G_VC, G_KB, G_VB, G_XN, G_ATTN = G_XN + 8, G_ACT = G_ATTN + 8, G_COUNT = G_ACT + 8 };
 
 struct LayerPtrs {
   const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
@@ -147,7 +146,16 @@ struct alignas(64) Plan {
   float* att_o;
   float2* att_ml;
   int* att_cnt;
-  size_t layers_off, maps_off;
+  // persistent forward kernel
+  CUtensorMap* d_maps;  // device copy of the tensor maps
+  LayerNorms* d_norms;  // device copy of the per-layer gains
+  int* phase_cnt;
+  int* exit_cnt;
+  float* ss;
+  int ss_ld, mega_slots, fwd_ck;
+  float* fwd_att_o;
+  float2* fwd_att_ml;
+  size_t layers_off, maps_off, norms_off;
   // profiling hook (host memory, written during the calls)
   void* const* trace_ev;
   int32_t* trace_kind;
@@ -162,6 +170,7 @@ struct alignas(64) Plan {
   CUtensorMap* lmap_mut(int l, int which) {
     return reinterpret_cast<CUtensorMap*>((char*)this + maps_off) + l * M_PER_LAYER + which;
   }
+  LayerNorms* norms_host() { return reinterpret_cast<LayerNorms*>((char*)this + norms_off); }
   const CUtensorMap& gmap(int which) const {
     return reinterpret_cast<const CUtensorMap*>((const char*)this + maps_off)[L * M_PER_LAYER + which];
   }
@@ -170,12 +179,16 @@ struct alignas(64) Plan {
   }
 };
 
-size_t plan_layout(int L, size_t* layers_off, size_t* maps_off) {
+size_t n_maps(int L) { return (size_t)L * M_PER_LAYER + G_COUNT; }
+
+size_t plan_layout(int L, size_t* layers_off, size_t* maps_off, size_t* norms_off) {
   size_t off = align_up(sizeof(Plan), 64);
   *layers_off = off;
   off = align_up(off + sizeof(LayerPtrs) * (size_t)L, 64);
   *maps_off = off;
-  off += sizeof(CUtensorMap) * (size_t)(L * M_PER_LAYER + G_COUNT);
+  off = align_up(off + sizeof(CUtensorMap) * n_maps(L), 64);
+  *norms_off = off;
+  off += sizeof(LayerNorms) * (size_t)L;
   return off + 64;  // slack for aligning the caller's buffer
 }
 
@@ -210,9 +223,19 @@ int attn_chunk_keys(int B, int Hkv, int row_tiles, int cap) {
 // workspace layout
 struct WsLayout {
   size_t status, h, xn, qbuf, attn, act, rope, amax, draft_ids, ar_ids, gemm_part, gemm_cnt, att_o, att_ml, att_cnt,
-      blk_k, blk_v, total;
-  int chunk_keys, attn_slots;
+      blk_k, blk_v, dev_maps, dev_norms, phase_cnt, ss, fwd_att_o, fwd_att_ml, total;
+  int chunk_keys, attn_slots, ss_ld, mega_slots;
 };
+
+// Attention slots of the persistent forward kernel for this batch and block limit
+// (0 when the kernel cannot run these sizes: more than 128 token rows or too many slots).
+int mega_slots(const orthrus_config* c, int B, int max_block) {
+  const int G = c->n_heads / c->n_kv_heads;
+  if (B * (max_block + 1) > 128 || c->d_model > 8192) return 0;
+  const int rt = (G * (max_block + 1) + 127) / 128;
+  const int slots = B * c->n_kv_heads * rt;
+  return slots <= kMaxSlots ? slots : 0;
+}
 
 int gemm_counter_count(const orthrus_config* c, int max_rows) {
   const int mt = (max_rows + 127) / 128;
@@ -260,6 +283,14 @@ WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows_r
   const size_t blk = (size_t)L * B * Hkv * max_block * d * 2;
   w.blk_k = take(blk);
   w.blk_v = take(blk);
+  w.dev_maps = take(sizeof(CUtensorMap) * ((size_t)L * M_PER_LAYER + G_COUNT));
+  w.dev_norms = take(sizeof(LayerNorms) * (size_t)L);
+  w.phase_cnt = take((size_t)(fwd_n_phases(L) + 1) * 4);
+  w.ss_ld = max_rows;
+  w.ss = take((size_t)(D / 128) * max_rows * 4);
+  w.mega_slots = mega_slots(c, B, max_block);
+  w.fwd_att_o = take((size_t)std::max(1, w.mega_slots) * kMaxChunks * 128 * d * 4);
+  w.fwd_att_ml = take((size_t)std::max(1, w.mega_slots) * kMaxChunks * 128 * 8);
   w.total = off;
   return w;
 }
@@ -331,6 +362,122 @@ GemmArgs base_gemm_args(const Plan* P) {
   a.tile_counter = P->gemm_cnt;
   a.status = P->status;
   return a;
+}
+
+// ---------------------------------------------------------------------------
+// persistent forward kernel (draft and verify views, at most 128 token rows)
+// ---------------------------------------------------------------------------
+// ORTHRUS_PERSISTENT=0 in the environment selects the per-op kernels instead.
+bool persistent_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("ORTHRUS_PERSISTENT");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* e = getenv(name);
+  return e && *e ? atoi(e) : dflt;
+}
+
+bool persistent_ok(const Plan* P, int Q) {
+  return persistent_enabled() && P->mega_slots > 0 && P->B * Q <= 128 && Q <= P->max_block + 1;
+}
+
+orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending, const int* draft, int* out_ids,
+                              float* logits, bool accept, int K, int* pending_out, int* accept_len, int* committed,
+                              cudaStream_t st) {
+  const orthrus_config& c = P->cfg;
+  FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.maps = P->d_maps;
+  a.norms = P->d_norms;
+  a.L = P->L;
+  a.D = c.d_model;
+  a.H = c.n_heads;
+  a.Hkv = c.n_kv_heads;
+  a.d = c.head_dim;
+  a.F = c.d_ff;
+  a.V = c.vocab;
+  a.G = c.n_heads / c.n_kv_heads;
+  a.qk_norm = c.qk_norm;
+  a.mask_id = c.mask_id;
+  a.eps = c.rms_eps;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
+  a.theta = (double)c.rope_theta;
+  a.view = view;
+  a.nb = P->B;
+  a.Q = Q;
+  a.M = P->B * Q;
+  a.Mt = round_up(a.M, 16);
+  a.mt_idx = a.Mt / 16 - 1;
+  const size_t stage = fwd_stage_bytes(a.Mt);
+  a.stages = (int)std::min<size_t>(kMaxStages, (kSmemLimit - fwd_fixed_smem(a.d)) / stage);
+  a.stages = std::max(2, std::min(a.stages, env_int("ORTHRUS_STAGES", a.stages)));
+  const size_t smem = fwd_fixed_smem(a.d) + (size_t)a.stages * stage;
+  a.cap = P->cap;
+  a.max_block = P->max_block;
+  a.batch = P->B;
+  const int sms = num_sms();
+  a.ck = P->fwd_ck;
+  a.pending = pending;
+  a.draft_ids = draft;
+  a.len = P->len;
+  a.embed = (const __nv_bfloat16*)P->embed;
+  a.final_norm = P->final_norm;
+  a.kc = P->kc;
+  a.vc = P->vc;
+  a.blk_k = P->blk_k;
+  a.blk_v = P->blk_v;
+  a.h = P->h;
+  a.xg = P->xn;
+  a.qbuf = P->qbuf;
+  a.attn = P->attn;
+  a.act = P->act;
+  a.rope = P->rope;
+  a.ss = P->ss;
+  a.ss_ld = P->ss_ld;
+  a.amax = P->amax;
+  a.out_ids = out_ids;
+  a.logits = logits;
+  a.partial = P->gemm_part;
+  a.tile_cnt = P->gemm_cnt;
+  a.phase_cnt = P->phase_cnt;
+  a.exit_cnt = P->exit_cnt;
+  a.att_o = P->fwd_att_o;
+  a.att_ml = P->fwd_att_ml;
+  a.status = P->status;
+  a.diag = P->status + 16;  // inside the status block of the workspace
+  a.accept = accept ? 1 : 0;
+  a.K = K;
+  a.pending_out = pending_out;
+  a.accept_len = accept_len;
+  a.committed = committed;
+
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(kFwdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (c.head_dim == 128) {
+    static bool set = false;
+    if (!set) set = set_smem_attr(forward_kernel<128>, kSmemLimit);
+    e = cudaLaunchKernelEx(&cfg, forward_kernel<128>, a);
+  } else {
+    static bool set = false;
+    if (!set) set = set_smem_attr(forward_kernel<64>, kSmemLimit);
+    e = cudaLaunchKernelEx(&cfg, forward_kernel<64>, a);
+  }
+  return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }
 
 // One forward over a block of Q rows for sequences [b0, b0+nb).
@@ -494,8 +641,8 @@ extern "C" {
 
 size_t orthrus_plan_bytes(const orthrus_config* cfg) {
   if (!config_ok(cfg)) return 0;
-  size_t a, b;
-  return plan_layout(cfg->n_layers, &a, &b);
+  size_t a, b, n;
+  return plan_layout(cfg->n_layers, &a, &b, &n);
 }
 
 static bool sizes_ok(const orthrus_config* cfg, int batch, int capacity, int max_block, int max_rows) {
@@ -528,8 +675,8 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   if (!cache->k || !cache->v || !cache->len) return ORTHRUS_ERR_ARG;
   if (!sizes_ok(cfg, cache->batch, cache->capacity, max_block, max_rows)) return ORTHRUS_ERR_ARG;
   const int L = cfg->n_layers;
-  size_t layers_off, maps_off;
-  if (plan_bytes < plan_layout(L, &layers_off, &maps_off)) return ORTHRUS_ERR_WORKSPACE;
+  size_t layers_off, maps_off, norms_off;
+  if (plan_bytes < plan_layout(L, &layers_off, &maps_off, &norms_off)) return ORTHRUS_ERR_WORKSPACE;
   const WsLayout wl = ws_layout(cfg, cache->batch, max_block, max_rows, cache->capacity);
   if (workspace_bytes < wl.total) return ORTHRUS_ERR_WORKSPACE;
   if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->mlp_norm || !w->w_qkv || !w->w_o ||
@@ -575,6 +722,19 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->att_cnt = (int*)(base + wl.att_cnt);
   P->blk_k = (__nv_bfloat16*)(base + wl.blk_k);
   P->blk_v = (__nv_bfloat16*)(base + wl.blk_v);
+  P->d_maps = (CUtensorMap*)(base + wl.dev_maps);
+  P->d_norms = (LayerNorms*)(base + wl.dev_norms);
+  P->phase_cnt = (int*)(base + wl.phase_cnt);
+  P->exit_cnt = P->phase_cnt + fwd_n_phases(L);
+  P->ss = (float*)(base + wl.ss);
+  P->ss_ld = wl.ss_ld;
+  P->mega_slots = wl.mega_slots;
+  // attention chunk of the persistent kernel: at most 16 chunks over the whole capacity
+  P->fwd_ck = std::max(64, round_up((P->cap + 15) / 16, 64));
+  P->fwd_ck = std::max(P->fwd_ck, round_up(env_int("ORTHRUS_ATT_CK", 0), 64));
+  P->fwd_att_o = (float*)(base + wl.fwd_att_o);
+  P->fwd_att_ml = (float2*)(base + wl.fwd_att_ml);
+  P->norms_off = norms_off;
   P->layers_off = layers_off;
   P->maps_off = maps_off;
 
@@ -603,6 +763,14 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
     ok = ok && map2d(P->lmap_mut(l, M_WDOWN), lp.w_down, F, D, 64, 128);
     ok = ok && map2d(P->lmap_mut(l, M_WDQKV), lp.wd_qkv, D, qkv_rows, 64, 128);
     ok = ok && map2d(P->lmap_mut(l, M_WDO), lp.wd_o, H * d, D, 64, 128);
+    ok = ok && map3d(P->lmap_mut(l, M_WGU3), lp.w_gu, D, F, 2, 64, 2);
+    LayerNorms& ln = P->norms_host()[l];
+    ln.attn_norm = lp.attn_norm;
+    ln.mlp_norm = lp.mlp_norm;
+    ln.q_norm = lp.q_norm;
+    ln.k_norm = lp.k_norm;
+    ln.wd_q_norm = lp.wd_q_norm;
+    ln.wd_k_norm = lp.wd_k_norm;
   }
   ok = ok && map2d(P->gmap_mut(G_LM), w->lm_head, D, V, 64, 128);
   const int rows = act_rows(max_rows);
@@ -617,8 +785,18 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   ok = ok && map3d(P->gmap_mut(G_VC), P->vc, d, P->cap, zc);
   ok = ok && map3d(P->gmap_mut(G_KB), P->blk_k, d, max_block, zc);
   ok = ok && map3d(P->gmap_mut(G_VB), P->blk_v, d, max_block, zc);
+  ok = ok && map3d(P->gmap_mut(G_KC64), P->kc, d, P->cap, zc, 64);
+  ok = ok && map3d(P->gmap_mut(G_VC64), P->vc, d, P->cap, zc, 64);
+  ok = ok && map3d(P->gmap_mut(G_KB64), P->blk_k, d, max_block, zc, 64);
+  ok = ok && map3d(P->gmap_mut(G_VB64), P->blk_v, d, max_block, zc, 64);
   if (!ok) return ORTHRUS_ERR_ARG;
   if (cudaMemsetAsync(workspace, 0, wl.total, (cudaStream_t)stream) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+  // the persistent kernel reads the tensor maps and norm gains from device memory
+  if (cudaMemcpyAsync(P->d_maps, &P->lmap(0, 0), sizeof(CUtensorMap) * n_maps(L), cudaMemcpyHostToDevice,
+                      (cudaStream_t)stream) != cudaSuccess ||
+      cudaMemcpyAsync(P->d_norms, P->norms_host(), sizeof(LayerNorms) * L, cudaMemcpyHostToDevice,
+                      (cudaStream_t)stream) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
   P->magic = kPlanMagic;
   return ORTHRUS_OK;
 }
@@ -656,6 +834,7 @@ orthrus_status orthrus_trace(void* plan, void* const* events, int32_t* kinds, in
 int32_t orthrus_decode_step_launches(const void* plan, int32_t K) {
   const Plan* P = plan_cast(plan);
   if (!P || K < 1 || K > P->max_block) return 0;
+  if (persistent_ok(P, K) && persistent_ok(P, K + 1)) return 2;
   const int per_forward = 1 + 7 * P->L + 3;
   return 2 * per_forward + 1;
 }
@@ -692,8 +871,15 @@ orthrus_status orthrus_draft_block(const void* plan, const int32_t* pending, int
                                    orthrus_stream stream) {
   const Plan* P = plan_cast(plan);
   if (!P || !pending || !draft || K < 1 || K > P->max_block) return ORTHRUS_ERR_ARG;
-  orthrus_status s = forward(P, BLOCK_DRAFT, 0, P->B, K, pending, nullptr, nullptr, 0, 0, true, false, draft, logits,
-                             (cudaStream_t)stream);
+  orthrus_status s;
+  if (persistent_ok(P, K)) {
+    mark(P, ORTHRUS_KIND_FORWARD, (cudaStream_t)stream);
+    s = launch_forward(P, VIEW_DRAFT, K, pending, nullptr, draft, logits, false, 0, nullptr, nullptr, nullptr,
+                       (cudaStream_t)stream);
+  } else {
+    s = forward(P, BLOCK_DRAFT, 0, P->B, K, pending, nullptr, nullptr, 0, 0, true, false, draft, logits,
+                (cudaStream_t)stream);
+  }
   mark(P, ORTHRUS_KIND_END, (cudaStream_t)stream);
   return s;
 }
@@ -702,8 +888,15 @@ orthrus_status orthrus_verify_block(const void* plan, const int32_t* pending, co
                                     int32_t* ar_argmax, float* logits, orthrus_stream stream) {
   const Plan* P = plan_cast(plan);
   if (!P || !pending || !ar_argmax || K < 0 || K > P->max_block || (K > 0 && !draft)) return ORTHRUS_ERR_ARG;
-  orthrus_status s = forward(P, BLOCK_VERIFY, 0, P->B, K + 1, pending, draft, nullptr, 0, 0, true, false, ar_argmax,
-                             logits, (cudaStream_t)stream);
+  orthrus_status s;
+  if (persistent_ok(P, K + 1)) {
+    mark(P, ORTHRUS_KIND_FORWARD, (cudaStream_t)stream);
+    s = launch_forward(P, VIEW_VERIFY, K + 1, pending, draft, ar_argmax, logits, false, K, nullptr, nullptr, nullptr,
+                       (cudaStream_t)stream);
+  } else {
+    s = forward(P, BLOCK_VERIFY, 0, P->B, K + 1, pending, draft, nullptr, 0, 0, true, false, ar_argmax, logits,
+                (cudaStream_t)stream);
+  }
   mark(P, ORTHRUS_KIND_END, (cudaStream_t)stream);
   return s;
 }
@@ -740,6 +933,13 @@ orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K
   if (planted && cudaMemcpyAsync(P->draft_ids, planted, sizeof(int) * P->B * K, cudaMemcpyDeviceToDevice, st) !=
                      cudaSuccess)
     return ORTHRUS_ERR_CUDA;
+  if (persistent_ok(P, K + 1)) {  // verify view with the greedy consensus fused into its last CTA
+    mark(P, ORTHRUS_KIND_FORWARD, st);
+    s = launch_forward(P, VIEW_VERIFY, K + 1, pending, P->draft_ids, P->ar_ids, nullptr, true, K, pending, accept_len,
+                       committed, st);
+    mark(P, ORTHRUS_KIND_END, st);
+    return s;
+  }
   s = orthrus_verify_block(plan, pending, P->draft_ids, K, P->ar_ids, nullptr, stream);
   if (s != ORTHRUS_OK) return s;
   return orthrus_accept_commit(plan, pending, P->draft_ids, P->ar_ids, K, accept_len, committed, 0, stream);

@@ -90,6 +90,92 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// Same wait, but it gives up early once the device status word holds an error
+// (another CTA has already failed): used by the persistent forward kernel, whose
+// roles would otherwise each sit out a full timeout after the first failure.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t parity, int* status) {
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 1023u) == 0u) {
+      if (*(volatile int*)status != 0) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        set_status(status, ORTHRUS_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Same as mbar_wait_abortable, but tells the two failures apart: 1 = phase
+// completed, 0 = gave up because the status word already held an error,
+// -1 = this wait ran out of time (ORTHRUS_ERR_TIMEOUT recorded).
+__device__ __forceinline__ int mbar_wait_code(uint64_t* bar, uint32_t parity, int* status) {
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i)
+    if (mbar_try_wait(bar, parity)) return 1;
+  const long long t0 = clock64();
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return 1;
+    if ((it & 1023u) == 0u) {
+      if (*(volatile int*)status != 0) return 0;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        set_status(status, ORTHRUS_ERR_TIMEOUT);
+        return -1;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// device-wide counters (release / acquire at GPU scope)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// generic-proxy global writes <-> later async-proxy (TMA) accesses
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void sleep_ns(uint32_t ns) { asm volatile("nanosleep.u32 %0;" ::"r"(ns)); }
+
+// Wait until *cnt >= target (acquire). False once the status word holds an
+// error or after about 2 s (then ORTHRUS_ERR_TIMEOUT is recorded).
+// 1 = reached, 0 = gave up because the status word holds an error, -1 = timed out here.
+__device__ __forceinline__ int wait_count_code(const int* cnt, int target, int* status) {
+  if (ld_acquire_gpu(cnt) >= target) return 1;
+  const long long t0 = clock64();
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    sleep_ns(64);
+    if (ld_acquire_gpu(cnt) >= target) return 1;
+    if ((it & 255u) == 0u) {
+      if (*(volatile int*)status != 0) return 0;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        set_status(status, ORTHRUS_ERR_TIMEOUT);
+        return -1;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_count(const int* cnt, int target, int* status) {
+  return wait_count_code(cnt, target, status) == 1;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (bulk tensor copies global -> shared, completion on an mbarrier)
 // ---------------------------------------------------------------------------
@@ -119,6 +205,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
 

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liborthrus.so")
 
 KIND_NAMES = ["embed", "rmsnorm", "gemm_qkv", "attention", "gemm_o", "gemm_gate_up", "gemm_down", "lm_head",
-              "argmax", "accept", "other", "end"]
+              "argmax", "accept", "other", "end", "forward"]
 
 OK, ERR_ARG, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_NAN, ERR_UNSUPPORTED, ERR_WORKSPACE = range(8)
 STATUS_NAMES = {0: "OK", 1: "ARG", 2: "CAPACITY", 3: "CUDA", 4: "TIMEOUT", 5: "NAN", 6: "UNSUPPORTED",
