@@ -70,7 +70,8 @@ constexpr int kMaxStages = 16;
 constexpr int kMaxSlots = 256;        // attention (sequence, kv head, row tile) slots per launch
 constexpr int kMaxChunks = 18;        // key chunks per slot (16 cache chunks + draft block + slack)
 constexpr int kCombineRows = 16;      // rows per merge unit
-constexpr int kScratchBytes = 17408;  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
+constexpr int kScratchBytes = 17408;
+constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
 
 struct LayerNorms {  // device-resident per-layer gains (fp32)
   const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
@@ -84,6 +85,7 @@ struct FwdArgs {
   double theta;
   int view;                  // VIEW_DRAFT / VIEW_VERIFY
   int nb, Q, M, Mt, mt_idx, stages, cap, max_block, batch;
+  int lookahead;             // weight tiles the weight producer loads ahead of a phase's input dependency
   int ck;                    // keys per attention chunk: fixed per plan (multiple of 64, >= capacity / 16),
                              // so a row's softmax runs over the same absolute key chunks whatever
                              // the block size: verify rows equal the plain AR rows bit for bit
@@ -112,6 +114,7 @@ struct FwdArgs {
   float2* att_ml;            // [kMaxSlots][kMaxChunks][128]
   int* status;
   int* diag;                 // [16] where the first timed-out wait gave up (nullable)
+  unsigned long long* tl;    // nullable [grid][phases][8] event times (profiling)
   // greedy consensus fused into the verify launch
   int accept, K;
   int* pending_out;          // [nb]
@@ -136,6 +139,22 @@ __device__ inline void fwd_diag(const FwdArgs& a, int code, int site, int p, int
   __threadfence();
 }
 
+// Phase timeline events (globaltimer, ns), per CTA and phase:
+//   0/1 weight producer first/last load issued, 2/3 activation producer dependency
+//   met / last load issued, 4/5 first MMA / last MMA commit, 6/7 epilogue
+//   dependency met / phase finished.
+//   8..13 (last epilogue segment of a projection phase): accumulator ready, partial
+//   stored, arrival counted, partials loaded, epilogue done, completion signalled.
+enum { TL_W0 = 0, TL_W1, TL_X0, TL_X1, TL_M0, TL_M1, TL_E0, TL_E1, TL_S_ACC, TL_S_PART, TL_S_CNT, TL_S_LOAD,
+       TL_S_EPI, TL_S_SIG, TL_R0, TL_R1, TL_EVENTS };
+__device__ __forceinline__ void tl_mark(const FwdArgs& a, int n_ph, int p, int ev) {
+  if (a.tl) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    a.tl[((size_t)blockIdx.x * n_ph + p) * TL_EVENTS + ev] = t;
+  }
+}
+
 __host__ __device__ inline int fwd_n_phases(int L) { return 2 + kPhasesPerLayer * L; }
 __host__ __device__ inline int fwd_phase_kind(int p, int L) {
   if (p == 0) return PH_EMBED;
@@ -149,7 +168,8 @@ __host__ __device__ inline int fwd_phase_layer(int p) { return (p - 1) / kPhases
 // staging, small per-CTA tables and the barriers.
 __host__ inline size_t fwd_fixed_smem(int d) {
   return 1024 /*align*/ + (size_t)128 * d * 2 /*Q*/ + kScratchBytes + 128 * 8 /*red*/ + 128 * 4 /*rstd*/ +
-         128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/;
+         128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/ +
+         kMaxGrid * 4 /*unit-range starts*/;
 }
 __host__ inline size_t fwd_stage_bytes(int Mt) { return 16384 + (size_t)Mt * 128; }
 
@@ -296,14 +316,17 @@ __device__ inline AttUnit att_unit(const FwdArgs& a, const FwdGeom& g, const int
 // Residual epilogue of the O and down projections on 32 token rows [m0, m0+32)
 // of one 128-column tile: h += v; xg = bf16(h * gamma_next); partial sum of h^2
 // over the tile's 128 columns per row -> ss[nt][m]. Thread = output column `row`.
+// With h_in_v the old h is already part of v (added by the contributor that holds
+// the tile's last k-chunk, early in its range, so no h load sits on the path).
 __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
-                                                   int m_valid, const float* gam, float* epi) {
+                                                   int m_valid, const float* gam, float* epi, bool h_in_v) {
   const int D = a.D;
   const int f = nt * 128 + row;
   const float gf = gam[f];
   float hv[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) hv[j] = (m0 + j < m_valid) ? __ldcg(a.h + (size_t)(m0 + j) * D + f) : 0.f;
+  for (int j = 0; j < 32; ++j)
+    hv[j] = (!h_in_v && m0 + j < m_valid) ? __ldcg(a.h + (size_t)(m0 + j) * D + f) : 0.f;
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     if (m0 + j < m_valid) {
@@ -331,9 +354,9 @@ __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float
 // normalised input first scale by rstd of the token row.
 __device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const GemmArgs& ga, int epi_kind, float* v, int row,
                                              int m0, int nt, int m_valid, float* epi, unsigned long long* red,
-                                             const float* rstd_s, const float* gam) {
+                                             const float* rstd_s, const float* gam, bool h_in_v = false) {
   if (epi_kind == EPI_RESID) {
-    fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam, epi);
+    fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam, epi, h_in_v);
     return;
   }
 #pragma unroll
@@ -402,7 +425,7 @@ template <int D_HEAD>
 __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeom& g, uint8_t* smem,
                                                   uint32_t stage_bytes, int S, uint8_t* scr,
                                                   unsigned long long* red, float* rstd_s, const int* lens_s,
-                                                  const int* slot_pre, uint64_t* accf, uint64_t* acce,
+                                                  const int* slot_pre, int* ust_s, uint64_t* accf, uint64_t* acce,
                                                   uint64_t* full, uint64_t* s_full, uint64_t* p_full,
                                                   uint64_t* o_full, uint64_t* t_done, int* flag,
                                                   uint32_t tmem_base, uint32_t tS, uint32_t tO) {
@@ -420,6 +443,8 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
   const int D = a.D;
   int seg = 0, ta = 0, it = 0, acq = -1, bc = 0;
   bool ok = true;
+  const uint64_t pol_keep = policy_evict_last();
+  const uint64_t pol_drop = policy_evict_first();
 
   // one thread waits, the result is shared by the four warps (rotating flag slots
   // keep a slow reader from seeing the next call's value)
@@ -446,9 +471,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
     }
     return r;
   };
+  // outputs of a completion unit written -> count it (the barrier orders the other
+  // threads' stores before thread 0's release, which is cumulative)
   auto signal = [&](int p) {
     fence_proxy_async_global();
-    __threadfence();
     named_bar_sync(1, 128);
     if (et == 0) red_release_gpu_add(a.phase_cnt + p, 1);
   };
@@ -473,6 +499,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       // ---------------- embedding rows ----------------
       const float* g0 = a.norms[0].attn_norm;
       const int parts = D / 128;
+      if (et == 0 && c < a.M) tl_mark(a, n_ph, p, TL_E0);
       for (int m = c; m < a.M; m += Gd) {
         const int bb = m / a.Q, i = m - bb * a.Q;
         int id;
@@ -510,10 +537,13 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       const long long u0 = unit_start(W, Gd, c), u1 = unit_start(W, Gd, c + 1);
       const int kc = gp.k_chunks;
       if (u0 == u1) continue;
+      // unit-range start of every CTA (W * Gd < 2^31 for every phase shape accepted)
+      for (int i = et; i <= Gd; i += 128) ust_s[i] = (int)(((long long)W * i) / Gd);
       if (!acquire_phase(dep)) {
         ok = false;
         break;
       }
+      if (et == 0) tl_mark(a, n_ph, p, TL_E0);
       if (kind == PH_QKV || kind == PH_GU || kind == PH_LM) {
         if (et < a.Mt) {
           float s = 0.f;
@@ -578,6 +608,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           ok = false;
           break;
         }
+        if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
         tc_fence_after();
         const int nt = t;
         const int m_valid = min(a.Mt, a.M);
@@ -592,63 +623,105 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acce[buf]);
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
           signal(p);
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
         } else {
+          // owner of unit u = the CTA whose non-empty range holds it (largest c with start <= u)
+          auto owner = [&](int uu) {
+            int lo = 0, hi = Gd - 1;
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (ust_s[mid] <= uu) lo = mid;
+              else hi = mid - 1;
+            }
+            return lo;
+          };
+          const int c_lo = owner(t * kc), c_hi = owner((t + 1) * kc - 1);
+          const bool add_h = gp.epi == EPI_RESID && c == c_hi;
           const int slot = 2 * c + (t == first_tile ? 0 : 1);
           float* part = a.partial + (size_t)slot * (128 * 128) + (size_t)row * a.Mt;
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
+            if (add_h) {
+              float hv[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                hv[j] = (m0 + j < m_valid) ? __ldcg(a.h + (size_t)(m0 + j) * D + nt * 128 + row) : 0.f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += hv[j];
+            }
             const int n4 = min(32, a.Mt - m0) / 4;
+            // partials stay in L2 (evict_last) while the weight stream passes through it
 #pragma unroll
             for (int qq = 0; qq < 8; ++qq)
               if (qq < n4)
-                __stcg(reinterpret_cast<float4*>(part + m0) + qq,
-                       make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]));
+                st_f4_hint(reinterpret_cast<float4*>(part + m0) + qq,
+                           make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]), pol_keep);
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acce[buf]);
-          // contributors: the CTAs with a non-empty unit range inside the tile (with
-          // fewer units than CTAs, CTAs between two owners may have none)
-          const int c_lo = unit_owner((long long)t * kc, W, Gd);
-          const int c_hi = unit_owner((long long)(t + 1) * kc - 1, W, Gd);
           int n_contrib = 0;
-          for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += unit_start(W, Gd, cc + 1) > unit_start(W, Gd, cc);
-          __threadfence();
+          for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += ust_s[cc + 1] > ust_s[cc];
           named_bar_sync(1, 128);
           bool last = false;
-          if (et == 0) last = atomicAdd(a.tile_cnt + t, 1) == n_contrib - 1;
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_PART);
+          if (et == 0) last = atom_add_acq_rel_gpu(a.tile_cnt + t, 1) == n_contrib - 1;
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_CNT);
           last = bcast(last);
           if (last) {
-            __threadfence();
             if (et == 0) a.tile_cnt[t] = 0;
             for (int m0 = 0; m0 < a.Mt; m0 += 32) {
               const int n4 = min(32, a.Mt - m0) / 4;
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = 0.f;
-              for (int cc = c_lo; cc <= c_hi; ++cc) {  // fixed k order
-                if (unit_start(W, Gd, cc + 1) == unit_start(W, Gd, cc)) continue;  // no units, no partial
-                const int ft = (int)(unit_start(W, Gd, cc) / kc);
-                const float4* pp = reinterpret_cast<const float4*>(
-                    a.partial + (size_t)(2 * cc + (t == ft ? 0 : 1)) * (128 * 128) + (size_t)row * a.Mt + m0);
-                float4 x[8];
+              int cc = c_lo;
+              while (cc <= c_hi) {
+                // up to four contributors per round, their loads all in flight together
+                int s0 = -1, s1 = -1, s2 = -1, s3 = -1;
+                for (int q = 0; q < 4 && cc <= c_hi; ++cc) {
+                  if (ust_s[cc + 1] > ust_s[cc]) {
+                    const int sl = 2 * cc + (ust_s[cc] / kc == t ? 0 : 1);
+                    if (q == 0) s0 = sl;
+                    else if (q == 1) s1 = sl;
+                    else if (q == 2) s2 = sl;
+                    else s3 = sl;
+                    ++q;
+                  }
+                }
+                float4 x[4][8];
 #pragma unroll
-                for (int qq = 0; qq < 8; ++qq) x[qq] = qq < n4 ? __ldcg(pp + qq) : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int q = 0; q < 4; ++q) {
+                  const int sl = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
+                  const float4* pp = reinterpret_cast<const float4*>(
+                      a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128) + (size_t)row * a.Mt + m0);
 #pragma unroll
-                for (int qq = 0; qq < 8; ++qq) {
-                  v[4 * qq] += x[qq].x;
-                  v[4 * qq + 1] += x[qq].y;
-                  v[4 * qq + 2] += x[qq].z;
-                  v[4 * qq + 3] += x[qq].w;
+                  for (int qq = 0; qq < 8; ++qq)
+                    x[q][qq] = (sl >= 0 && qq < n4) ? ld_f4_hint(pp + qq, pol_drop) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {  // fixed k order within and across rounds
+#pragma unroll
+                  for (int qq = 0; qq < 8; ++qq) {
+                    v[4 * qq] += x[q][qq].x;
+                    v[4 * qq + 1] += x[q][qq].y;
+                    v[4 * qq + 2] += x[q][qq].z;
+                    v[4 * qq + 3] += x[q][qq].w;
+                  }
                 }
               }
-              fwd_epilogue(a, ga, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
+              fwd_epilogue(a, ga, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
             }
+            if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
             signal(p);
+            if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
           }
         }
       }
       it += (int)(u1 - u0);
+      if (et == 0) tl_mark(a, n_ph, p, TL_E1);
     } else if (kind == PH_ATTN) {
       // ---------------- block attention (thread = query row of the tile) ----------------
       if (c >= g.att_units) continue;
@@ -656,6 +729,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         ok = false;
         break;
       }
+      if (et == 0) tl_mark(a, n_ph, p, TL_E0);
       for (int u = c; ok && u < g.att_units; u += Gd) {
         const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
         const int grow = t.r * 128 + row;
@@ -772,6 +846,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         signal(p);
       }
+      if (et == 0) tl_mark(a, n_ph, p, TL_E1);
     } else if (kind == PH_COMBINE) {
       // ---------------- merge of key-chunk partials ----------------
       if (c >= g.comb_units) continue;
@@ -779,6 +854,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         ok = false;
         break;
       }
+      if (et == 0) tl_mark(a, n_ph, p, TL_E0);
       constexpr int per = d / 8;  // columns per thread
       for (int u = c; u < g.comb_units; u += Gd) {
         const int slot = u / (128 / kCombineRows), grp = u % (128 / kCombineRows);
@@ -822,6 +898,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         signal(p);
       }
+      if (et == 0) tl_mark(a, n_ph, p, TL_E1);
     }
   }
 }
@@ -845,7 +922,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   float* rstd_s = (float*)(red + 128);
   int* lens_s = (int*)(rstd_s + 128);
   int* slot_pre = lens_s + 128;
-  uint64_t* bars = (uint64_t*)(((uintptr_t)(slot_pre + kMaxSlots + 1) + 7) & ~(uintptr_t)7);
+  int* ust_s = slot_pre + kMaxSlots + 1;  // [grid + 1] unit-range starts of the current phase
+  uint64_t* bars = (uint64_t*)(((uintptr_t)(ust_s + kMaxGrid) + 7) & ~(uintptr_t)7);
   uint64_t* full = bars;
   uint64_t* empty = bars + kMaxStages;
   uint64_t* accf = bars + 2 * kMaxStages;  // [2]
@@ -954,6 +1032,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
           const long long W = gp.units;
           const long long u0 = unit_start(W, Gd, c), u1 = unit_start(W, Gd, c + 1);
           const int kc = gp.k_chunks;
+          if (u0 < u1 && wprod) tl_mark(a, n_ph, p, TL_W0);
           for (long long u = u0; u < u1; ++u, ++it) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -966,6 +1045,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
             const int t = (int)(u / kc), k = (int)(u - (long long)t * kc);
             uint8_t* st = stage_ptr(s);
             if (wprod) {
+              // run ahead into a phase whose input is not ready by at most `lookahead` tiles
+              if (u - u0 >= a.lookahead && !dep_ready(dep)) {
+                ok = false;
+                break;
+              }
               mbar_arrive_expect_tx(&full[s], 16384u);
               if (gp.gu) tma_load_3d_hint(st, gp.mw, &full[s], k * 64, t * 64, 0, pol_w);  // 64 gate + 64 up rows
               else tma_load_2d_hint(st, gp.mw, &full[s], k * 64, t * 128, pol_w);
@@ -974,11 +1058,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 ok = false;
                 break;
               }
+              if (u == u0) tl_mark(a, n_ph, p, TL_X0);
               mbar_arrive_expect_tx(&full[s], x_bytes);
               tma_load_2d(st + 16384, gp.mx, &full[s], k * 64, 0);
             }
             last_ph[s] = (int)ph;
           }
+          if (u0 < u1) tl_mark(a, n_ph, p, wprod ? TL_W1 : TL_X1);
         } else if (kind == PH_ATTN) {
           for (int u = c; ok && u < g.att_units; u += Gd, ++qu) {
             const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
@@ -1072,6 +1158,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 ok = false;
                 break;
               }
+              if (u == u0) tl_mark(a, n_ph, p, TL_M0);
               tc_fence_after();
               const uint32_t wa = smem_u32(stage_ptr(s));
               const uint32_t xa = wa + 16384;
@@ -1085,6 +1172,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
             mma_commit(&accf[buf]);
             ++seg;
           }
+          if (u0 < u1) tl_mark(a, n_ph, p, TL_M1);
         } else if (kind == PH_ATTN) {
           const uint32_t qa = smem_u32(sQ);
           for (int u = c; ok && u < g.att_units; u += Gd, ++qu) {
@@ -1146,7 +1234,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
     }
   } else {
     // ======================= epilogue warps =======================
-    fwd_epilogue_role<D_HEAD>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, accf, acce, full,
+    fwd_epilogue_role<D_HEAD>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, ust_s, accf, acce, full,
                               s_full, p_full, o_full, t_done, flag, tmem_base, tS, tO);
   }
 

@@ -161,6 +161,8 @@ struct alignas(64) Plan {
   int32_t* trace_kind;
   int32_t trace_cap;
   int32_t* trace_count;
+  unsigned long long* timeline;  // device, nullable: per-CTA phase events of the persistent kernel
+  size_t timeline_bytes;
 
   const LayerPtrs& layer(int l) const { return reinterpret_cast<const LayerPtrs*>((const char*)this + layers_off)[l]; }
   LayerPtrs& layer(int l) { return reinterpret_cast<LayerPtrs*>((char*)this + layers_off)[l]; }
@@ -422,6 +424,7 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.batch = P->B;
   const int sms = num_sms();
   a.ck = P->fwd_ck;
+  a.lookahead = std::max(0, env_int("ORTHRUS_LOOKAHEAD", a.stages));
   a.pending = pending;
   a.draft_ids = draft;
   a.len = P->len;
@@ -450,6 +453,8 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.att_ml = P->fwd_att_ml;
   a.status = P->status;
   a.diag = P->status + 16;  // inside the status block of the workspace
+  const size_t tl_need = (size_t)num_sms() * fwd_n_phases(P->L) * TL_EVENTS * 8;
+  a.tl = (P->timeline && P->timeline_bytes >= tl_need) ? P->timeline : nullptr;
   a.accept = accept ? 1 : 0;
   a.K = K;
   a.pending_out = pending_out;
@@ -828,6 +833,20 @@ orthrus_status orthrus_trace(void* plan, void* const* events, int32_t* kinds, in
   P->trace_kind = kinds;
   P->trace_cap = capacity;
   P->trace_count = count;
+  return ORTHRUS_OK;
+}
+
+size_t orthrus_timeline_bytes(const void* plan) {
+  const Plan* P = plan_cast(plan);
+  return P ? (size_t)num_sms() * fwd_n_phases(P->L) * TL_EVENTS * 8 : 0;
+}
+
+orthrus_status orthrus_timeline(void* plan, void* device_buf, size_t bytes) {
+  Plan* P = plan_cast(plan);
+  if (!P) return ORTHRUS_ERR_ARG;
+  if (device_buf && bytes < orthrus_timeline_bytes(plan)) return ORTHRUS_ERR_WORKSPACE;
+  P->timeline = (unsigned long long*)device_buf;
+  P->timeline_bytes = device_buf ? bytes : 0;
   return ORTHRUS_OK;
 }
 

@@ -66,6 +66,8 @@ SIGNATURES = [
     ("orthrus_clear_status", _I32, [_VP, _VP]),
     ("orthrus_decode_step_launches", _I32, [_VP, _I32]),
     ("orthrus_trace", _I32, [_VP, _VP, _VP, _I32, _VP]),
+    ("orthrus_timeline_bytes", _SZ, [_VP]),
+    ("orthrus_timeline", _I32, [_VP, _VP, _SZ]),
     ("orthrus_prefill", _I32, [_VP, _VP, _VP, _I32, _VP, _VP]),
     ("orthrus_draft_block", _I32, [_VP, _VP, _I32, _VP, _VP, _VP]),
     ("orthrus_verify_block", _I32, [_VP, _VP, _VP, _I32, _VP, _VP, _VP]),
@@ -259,6 +261,17 @@ class DeviceModel:
             _check("orthrus_trace", load().orthrus_trace(self.plan, None, None, 0, None))
         else:
             _check("orthrus_trace", load().orthrus_trace(self.plan, events, kinds, len(events), count))
+
+    def timeline(self, buf):
+        """buf: device uint8/int64 tensor of timeline_bytes() bytes, or None to stop."""
+        if buf is None:
+            _check("orthrus_timeline", load().orthrus_timeline(self.plan, None, 0))
+        else:
+            _check("orthrus_timeline",
+                   load().orthrus_timeline(self.plan, _ptr(buf), buf.numel() * buf.element_size()))
+
+    def timeline_bytes(self) -> int:
+        return load().orthrus_timeline_bytes(self.plan)
 
     def read_status(self) -> int:
         return int(self.status.item())
