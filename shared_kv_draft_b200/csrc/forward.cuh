@@ -70,8 +70,8 @@ constexpr int kMaxStages = 16;
 constexpr int kMaxSlots = 256;        // attention (sequence, kv head, row tile) slots per launch
 constexpr int kMaxChunks = 18;        // key chunks per slot (16 cache chunks + draft block + slack)
 constexpr int kCombineRows = 16;      // rows per merge unit
-constexpr int kScratchBytes = 17408;
-constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
+constexpr int kScratchBytes = 17408;  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
+constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers
 
 struct LayerNorms {  // device-resident per-layer gains (fp32)
   const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
@@ -350,18 +350,99 @@ __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float
   named_bar_sync(1, 128);
 }
 
+// Per-phase state of the q/k/v projection epilogue: destination of the block's
+// K/V and the q/k RMSNorm gains of this lane (element lane + 32 k of a head).
+struct QkvCtx {
+  __nv_bfloat16 *kdst, *vdst;
+  int kv_stride;
+  float gq[4], gk[4];
+};
+
+// q/k/v epilogue on 32 token rows [m0, m0+32) of one 128-row tile (one head at
+// d = 128, two at d = 64): per-head RMSNorm of q and k, rotate-half RoPE at the
+// row's absolute position, bf16 store of q (qbuf) and of k, v (cache slot len+i
+// in the verify view, block-scratch row i in the draft view). Warp ew handles
+// token rows ew, ew+4, ...; lane holds elements lane + 32 k of the head. The RoPE
+// factors of all its rows are loaded before the staging barrier (one round trip).
+template <int D_HEAD>
+__device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx& q, const float* v, int row, int m0,
+                                                 int nt, int m_valid, float* epi, const int* lens_s) {
+  constexpr int d = D_HEAD, nper = d / 32, half = d / 2;
+  const int lane = threadIdx.x & 31, ew = (threadIdx.x >> 5) - 2;
+  float2 cs[8][nper / 2];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int m = m0 + ew + 4 * r;
+#pragma unroll
+    for (int k = 0; k < nper / 2; ++k)
+      cs[r][k] = m < m_valid ? __ldcg(a.rope + (size_t)m * half + lane + 32 * k) : make_float2(1.f, 0.f);
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+  named_bar_sync(1, 128);
+  const int G = a.H / a.Hkv;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int j = ew + 4 * r, m = m0 + j;
+    if (m >= m_valid) break;
+    const int bb = m / a.Q, i = m - bb * a.Q;
+#pragma unroll
+    for (int hl = 0; hl < 128 / d; ++hl) {
+      const int hh = (nt * 128) / d + hl;  // head index in the fused q|k|v rows
+      const int kind = hh < a.H ? 0 : (hh < a.H + a.Hkv ? 1 : 2);
+      float x[nper];
+#pragma unroll
+      for (int k = 0; k < nper; ++k) x[k] = epi[j * kEpiStride + hl * d + lane + 32 * k];
+      if (kind < 2) {
+        if (a.qk_norm) {
+          float ss = 0.f;
+#pragma unroll
+          for (int k = 0; k < nper; ++k) ss += x[k] * x[k];
+          ss = warp_sum(ss);
+          const float rr = rsqrtf(ss / (float)d + a.eps);
+#pragma unroll
+          for (int k = 0; k < nper; ++k) x[k] = x[k] * rr * (kind == 0 ? q.gq[k] : q.gk[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < nper / 2; ++k) {  // element e pairs with e + d/2
+          const float x1 = x[k], x2 = x[k + nper / 2];
+          x[k] = x1 * cs[r][k].x - x2 * cs[r][k].y;
+          x[k + nper / 2] = x2 * cs[r][k].x + x1 * cs[r][k].y;
+        }
+      }
+      if (kind == 0) {
+        const int kvh = hh / G, g = hh - kvh * G;
+        __nv_bfloat16* dst = a.qbuf + ((size_t)(bb * a.Hkv + kvh) * (a.Q * G) + i * G + g) * d;
+#pragma unroll
+        for (int k = 0; k < nper; ++k) dst[lane + 32 * k] = __float2bfloat16(x[k]);
+      } else {
+        const int kvh = hh - a.H - (kind == 2 ? a.Hkv : 0);
+        const int slot = a.view == VIEW_DRAFT ? i : lens_s[bb] + i;
+        if (slot >= 0 && slot < q.kv_stride) {
+          __nv_bfloat16* dst = (kind == 1 ? q.kdst : q.vdst) + ((size_t)(bb * a.Hkv + kvh) * q.kv_stride + slot) * d;
+#pragma unroll
+          for (int k = 0; k < nper; ++k) dst[lane + 32 * k] = __float2bfloat16(x[k]);
+        }
+      }
+    }
+  }
+  named_bar_sync(1, 128);
+}
+
 // Epilogue of one 32-row group for the GEMM phase kinds. Consumers of a
 // normalised input first scale by rstd of the token row.
-__device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const GemmArgs& ga, int epi_kind, float* v, int row,
-                                             int m0, int nt, int m_valid, float* epi, unsigned long long* red,
-                                             const float* rstd_s, const float* gam, bool h_in_v = false) {
+template <int D_HEAD>
+__device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const GemmArgs& ga, const QkvCtx& qc, const int* lens_s,
+                                             int epi_kind, float* v, int row, int m0, int nt, int m_valid, float* epi,
+                                             unsigned long long* red, const float* rstd_s, const float* gam,
+                                             bool h_in_v = false) {
   if (epi_kind == EPI_RESID) {
     fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam, epi, h_in_v);
     return;
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] *= rstd_s[m0 + j];
-  if (epi_kind == EPI_QKV) epilogue_group<EPI_QKV>(ga, v, row, m0, 0, nt, m_valid, epi, red);
+  if (epi_kind == EPI_QKV) fwd_qkv_epilogue<D_HEAD>(a, qc, v, row, m0, nt, m_valid, epi, lens_s);
   else if (epi_kind == EPI_SWIGLU) epilogue_group<EPI_SWIGLU>(ga, v, row, m0, 0, nt, m_valid, epi, red);
   else epilogue_group<EPI_ARGMAX>(ga, v, row, m0, 0, nt, m_valid, epi, red);
 }
@@ -564,32 +645,29 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       ga.logits = a.logits;
       ga.ld_logits = a.V;
       const float* gam = nullptr;
+      QkvCtx qc;
+      qc.kdst = qc.vdst = nullptr;
+      qc.kv_stride = 0;
       if (kind == PH_QKV) {
         const bool dv = a.view == VIEW_DRAFT;
-        QkvEpi& q = ga.qkv;
-        q.H = a.H;
-        q.Hkv = a.Hkv;
-        q.d = d;
-        q.Q = a.Q;
-        q.b0 = 0;
-        q.qk_norm = a.qk_norm;
-        q.mode = a.view;
-        q.eps = a.eps;
-        q.gq = dv ? a.norms[l].wd_q_norm : a.norms[l].q_norm;
-        q.gk = dv ? a.norms[l].wd_k_norm : a.norms[l].k_norm;
-        q.rope = a.rope;
-        q.len = a.len;
-        q.qbuf = a.qbuf;
+        const float* gq = dv ? a.norms[l].wd_q_norm : a.norms[l].q_norm;
+        const float* gk = dv ? a.norms[l].wd_k_norm : a.norms[l].k_norm;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const bool in = a.qk_norm && k < d / 32;
+          qc.gq[k] = in ? gq[lane + 32 * k] : 1.f;
+          qc.gk[k] = in ? gk[lane + 32 * k] : 1.f;
+        }
         if (dv) {
           const size_t lo = (size_t)l * a.batch * a.Hkv * a.max_block * d;
-          q.kdst = a.blk_k + lo;
-          q.vdst = a.blk_v + lo;
-          q.kv_stride = a.max_block;
+          qc.kdst = a.blk_k + lo;
+          qc.vdst = a.blk_v + lo;
+          qc.kv_stride = a.max_block;
         } else {
           const size_t lo = (size_t)l * a.batch * a.Hkv * a.cap * d;
-          q.kdst = a.kc + lo;
-          q.vdst = a.vc + lo;
-          q.kv_stride = a.cap;
+          qc.kdst = a.kc + lo;
+          qc.vdst = a.vc + lo;
+          qc.kv_stride = a.cap;
         }
       } else if (kind == PH_O) {
         gam = a.norms[l].mlp_norm;
@@ -618,7 +696,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         if (whole) {
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
-            fwd_epilogue(a, ga, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
+            fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
           }
           tc_fence_before();
           __syncwarp();
@@ -712,7 +790,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                   }
                 }
               }
-              fwd_epilogue(a, ga, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
+              fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
             }
             if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
             signal(p);

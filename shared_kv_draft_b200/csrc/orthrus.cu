@@ -416,7 +416,9 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.Mt = round_up(a.M, 16);
   a.mt_idx = a.Mt / 16 - 1;
   const size_t stage = fwd_stage_bytes(a.Mt);
-  a.stages = (int)std::min<size_t>(kMaxStages, (kSmemLimit - fwd_fixed_smem(a.d)) / stage);
+  // 6 stages (about 96 KB of weight tiles in flight per SM) measured fastest; deeper
+  // rings put more requests in flight than HBM serves efficiently
+  a.stages = (int)std::min<size_t>(6, (kSmemLimit - fwd_fixed_smem(a.d)) / stage);
   a.stages = std::max(2, std::min(a.stages, env_int("ORTHRUS_STAGES", a.stages)));
   const size_t smem = fwd_fixed_smem(a.d) + (size_t)a.stages * stage;
   a.cap = P->cap;
