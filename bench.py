@@ -19,6 +19,7 @@ L2, so no L2 flush is needed between steps. Prints ONE JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import ctypes as C
 import json
 import os
@@ -51,6 +52,9 @@ WORKLOADS = {
     "qwen3_8b_b1_k32": dict(shape=synth.QWEN3_8B, batch=1, prompt=512, gen=1024, K=32, mean_accept=6.0,
                             steps=147),
     "tiny_b1_k8": dict(shape=synth.TINY, batch=1, prompt=64, gen=128, K=8, mean_accept=3.0, steps=32),
+    # two layers of the Qwen3-8B shape (same kernels, about 2 GB of weights): the small case for profiling
+    "qwen3_8b_2layer_b1_k32": dict(shape=dataclasses.replace(synth.QWEN3_8B, n_layers=2, name="qwen3_8b_2layer"),
+                                   batch=1, prompt=512, gen=1024, K=32, mean_accept=6.0, steps=40),
 }
 
 
