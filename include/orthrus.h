@@ -262,6 +262,26 @@ size_t orthrus_linear_workspace_bytes(int32_t M, int32_t N, int32_t Kd);
 orthrus_status orthrus_linear(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t Kd,
                               void* workspace, size_t workspace_bytes, int32_t* status, orthrus_stream stream);
 
+/* Allocation-free variant of orthrus_linear. This entry point has no
+ * counterpart in the paper; it exists for callers that cannot allocate device
+ * memory, such as a plugin or custom-operator interface that is handed only its
+ * input and output buffers by a host framework owning all device memory, or a
+ * runtime that works inside a fixed, pre-reserved memory budget.
+ * Same operation and arguments as orthrus_linear, without the workspace: the
+ * scratch (split-tile partial sums and tile counters) lives in a static device
+ * array of 4 MiB + 64 KiB inside the library, which every GPU that loads the
+ * library holds until the process exits. The call allocates nothing.
+ * Limits: (M+127)/128 * N/128 <= 16384 weight tiles, else ORTHRUS_ERR_WORKSPACE;
+ * the GEMM runs on at most 32 CTAs so the partial sums fit the array.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one array and it keeps the previous call's
+ * contents (the call clears the tile counters itself): calls that overlap on the
+ * GPU (different streams, or concurrent host threads) race and must not be
+ * issued. status: device int32 or NULL. */
+orthrus_status orthrus_linear_noalloc(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t Kd,
+                                      int32_t* status, orthrus_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

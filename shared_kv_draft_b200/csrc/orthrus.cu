@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <utility>
 
 #include "attention.cuh"
@@ -1071,3 +1072,85 @@ orthrus_status orthrus_linear(const void* X, const void* W, float* Y, int32_t M,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// orthrus_linear_noalloc: orthrus_linear with its scratch in a static device array
+// ---------------------------------------------------------------------------
+// Scratch of the stream-K GEMM: partial sums of split weight tiles (one 128 x 128
+// fp32 slot pair per CTA) and the tiles' arrival counters. The grid is capped at
+// kNoAllocCtas CTAs so the partial slots fit; the counters cover kNoAllocTiles
+// tiles. Every GPU that loads the library holds this array until the process exits.
+namespace {
+constexpr int kNoAllocCtas = 32;
+constexpr size_t kNoAllocPartialBytes = (size_t)2 * kNoAllocCtas * 128 * 128 * 4;  // 4 MiB
+constexpr int kNoAllocTiles = 16384;
+constexpr size_t kNoAllocBytes = kNoAllocPartialBytes + (size_t)kNoAllocTiles * 4;  // 4 MiB + 64 KiB
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_linear_scratch[kNoAllocBytes];
+
+namespace {
+// Device address of g_linear_scratch on the current device, looked up once per
+// device (host code cannot use the symbol itself as a device address).
+void* linear_scratch_address() {
+  static std::mutex mu;
+  static void* addr[256] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || !p) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+template <int EPI>
+cudaError_t launch_gemm_capped(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs a, int N, int Kd, int M,
+                               int max_ctas, cudaStream_t st) {
+  a.N = N;
+  a.Kd = Kd;
+  a.M = M;
+  a.m_tiles = (M + 127) / 128;
+  a.Mt = a.m_tiles > 1 ? 128 : round_up(std::max(M, 1), 16);
+  a.mt_alloc = std::max(32, next_pow2(a.Mt));
+  a.n_tiles = N / 128;
+  a.k_chunks = Kd / 64;
+  a.total_units = (long long)a.m_tiles * a.n_tiles * a.k_chunks;
+  const int G = (int)std::min<long long>(std::min(num_sms(), max_ctas), a.total_units);
+  const size_t fixed = gemm_smem_bytes(a.Mt, 0);
+  const size_t stage = 16384 + (size_t)a.Mt * 128;
+  a.stages = (int)std::min<size_t>(12, (kSmemLimit - fixed) / stage);
+  const size_t smem = gemm_smem_bytes(a.Mt, a.stages);
+  static bool attr = false;
+  if (!attr) attr = set_smem_attr(gemm_kernel<EPI>, kSmemLimit);
+  return launch(gemm_kernel<EPI>, dim3(G), dim3(kGemmThreads), smem, st, tmW, tmX, a);
+}
+}  // namespace
+
+extern "C" orthrus_status orthrus_linear_noalloc(const void* X, const void* W, float* Y, int32_t M, int32_t N,
+                                                 int32_t Kd, int32_t* status, orthrus_stream stream) {
+  if (!X || !W || !Y) return ORTHRUS_ERR_ARG;
+  if (M < 1 || N < 128 || N % 128 || Kd < 64 || Kd % 64) return ORTHRUS_ERR_UNSUPPORTED;
+  const long long tiles = (long long)((M + 127) / 128) * (N / 128);
+  if (tiles > kNoAllocTiles) return ORTHRUS_ERR_WORKSPACE;  // beyond the static scratch
+  if (!encode_fn()) return ORTHRUS_ERR_CUDA;
+  char* base = (char*)linear_scratch_address();
+  if (!base) return ORTHRUS_ERR_CUDA;
+  int* cnt = (int*)(base + kNoAllocPartialBytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  // the array keeps the previous call's contents: the arrival counters must start at zero
+  if (cudaMemsetAsync(cnt, 0, (size_t)tiles * 4, st) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+  CUtensorMap tw, tx;
+  if (!map2d(&tw, W, Kd, N, 64, 128) || !map2d(&tx, X, Kd, M, 64, 16 * (mt_index(M) + 1))) return ORTHRUS_ERR_ARG;
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.partial = (float*)base;
+  a.tile_counter = cnt;
+  a.status = status;
+  a.out_f32 = Y;
+  a.ld_out = N;
+  return launch_gemm_capped<EPI_STORE>(tw, tx, a, N, Kd, M, kNoAllocCtas, st) == cudaSuccess ? ORTHRUS_OK
+                                                                                            : ORTHRUS_ERR_CUDA;
+}

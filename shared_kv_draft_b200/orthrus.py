@@ -78,6 +78,7 @@ SIGNATURES = [
                                  _VP, _SZ, _VP, _VP]),
     ("orthrus_linear_workspace_bytes", _SZ, [_I32, _I32, _I32]),
     ("orthrus_linear", _I32, [_VP, _VP, _VP, _I32, _I32, _I32, _VP, _SZ, _VP, _VP]),
+    ("orthrus_linear_noalloc", _I32, [_VP, _VP, _VP, _I32, _I32, _I32, _VP, _VP]),
 ]
 
 _lib = None
@@ -161,6 +162,15 @@ def linear(X, W, Y, workspace, status, stream=None):
     code = lib.orthrus_linear(_ptr(X), _ptr(W), _ptr(Y), M, N, Kd, _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
     _check("orthrus_linear", code)
+
+
+def linear_noalloc(X, W, Y, status=None, stream=None):
+    """orthrus_linear without a workspace: scratch in the library's static device array."""
+    lib = load()
+    M, Kd = X.shape
+    N = W.shape[0]
+    code = lib.orthrus_linear_noalloc(_ptr(X), _ptr(W), _ptr(Y), M, N, Kd, _ptr(status), _stream(stream))
+    _check("orthrus_linear_noalloc", code)
 
 
 def linear_workspace_bytes(M, N, Kd) -> int:
