@@ -42,9 +42,27 @@
 namespace orthrus {
 
 // tensor-map indices: per layer, then global
-// M_WGU3 views W_gate_up as [2][d_ff][d_model] so one box brings 64 gate rows and the
-// 64 matching up rows (one 16 KB TMA copy instead of two 8 KB ones).
-enum { M_WQKV = 0, M_WO, M_WGU, M_WDOWN, M_WDQKV, M_WDO, M_WGU3, M_PER_LAYER };
+// The persistent kernel reads every projection through a 3-D view (64 columns, rows,
+// k chunk of 64) with strides (row, 128 bytes): one 32 KB box brings two consecutive
+// 64-wide k chunks of 128 rows (256 contiguous bytes per row), which streams about
+// 10% faster than two 16 KB boxes. M_WGU4 adds the gate/up half as a 4th dimension,
+// so a box holds, per k chunk, 64 gate rows and the 64 matching up rows.
+// The per-op kernels use the 2-D maps (M_WQKV .. M_WDO).
+enum {
+  M_WQKV = 0,
+  M_WO,
+  M_WGU,
+  M_WDOWN,
+  M_WDQKV,
+  M_WDO,
+  M_WQKV3,
+  M_WO3,
+  M_WDOWN3,
+  M_WDQKV3,
+  M_WDO3,
+  M_WGU4,
+  M_PER_LAYER
+};
 // activation maps exist for every token-tile height Mt = 16, 32, ..., 128 (index Mt/16 - 1)
 enum {
   G_LM = 0,
@@ -60,7 +78,11 @@ enum {
   G_XN,
   G_ATTN = G_XN + 8,
   G_ACT = G_ATTN + 8,
-  G_COUNT = G_ACT + 8
+  G_LM3 = G_ACT + 8,  // 3-D views of the LM head and of the activations (k-pair boxes)
+  G_XN3,
+  G_ATTN3 = G_XN3 + 8,
+  G_ACT3 = G_ATTN3 + 8,
+  G_COUNT = G_ACT3 + 8
 };
 
 enum PhaseKind : int { PH_EMBED = 0, PH_QKV, PH_ATTN, PH_COMBINE, PH_O, PH_GU, PH_DOWN, PH_LM };
@@ -171,7 +193,8 @@ __host__ inline size_t fwd_fixed_smem(int d) {
          128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/ +
          kMaxGrid * 4 /*unit-range starts*/;
 }
-__host__ inline size_t fwd_stage_bytes(int Mt) { return 16384 + (size_t)Mt * 128; }
+// ring stage: 32 KB weight box (128 rows x two k chunks) + activation box (Mt rows x two k chunks)
+__host__ inline size_t fwd_stage_bytes(int Mt) { return 32768 + (size_t)Mt * 256; }
 
 // Shared state every role derives identically at kernel start.
 struct FwdGeom {
@@ -186,7 +209,7 @@ struct FwdGeom {
 // GEMM phase description
 struct GemmPhase {
   int epi;            // EPI_QKV / EPI_RESID / EPI_SWIGLU / EPI_ARGMAX
-  int n_tiles, k_chunks;
+  int n_tiles, k_chunks;  // k_chunks: 128-wide k units per tile (each a pair of 64-wide chunks)
   long long units;
   const CUtensorMap* mw;
   const CUtensorMap* mx;
@@ -202,34 +225,34 @@ __device__ inline GemmPhase gemm_phase(const FwdArgs& a, int kind, int l) {
   if (kind == PH_QKV) {
     g.epi = EPI_QKV;
     g.n_tiles = (a.H + 2 * a.Hkv) * a.d / 128;
-    g.k_chunks = a.D / 64;
-    g.mw = lm + (draft ? M_WDQKV : M_WQKV);
-    g.mx = gm + G_XN + a.mt_idx;
+    g.k_chunks = a.D / 128;
+    g.mw = lm + (draft ? M_WDQKV3 : M_WQKV3);
+    g.mx = gm + G_XN3 + a.mt_idx;
   } else if (kind == PH_O) {
     g.epi = EPI_RESID;
     g.n_tiles = a.D / 128;
-    g.k_chunks = a.H * a.d / 64;
-    g.mw = lm + (draft ? M_WDO : M_WO);
-    g.mx = gm + G_ATTN + a.mt_idx;
+    g.k_chunks = a.H * a.d / 128;
+    g.mw = lm + (draft ? M_WDO3 : M_WO3);
+    g.mx = gm + G_ATTN3 + a.mt_idx;
   } else if (kind == PH_GU) {
     g.epi = EPI_SWIGLU;
     g.n_tiles = a.F / 64;
-    g.k_chunks = a.D / 64;
-    g.mw = lm + M_WGU3;
-    g.mx = gm + G_XN + a.mt_idx;
+    g.k_chunks = a.D / 128;
+    g.mw = lm + M_WGU4;
+    g.mx = gm + G_XN3 + a.mt_idx;
     g.gu = 1;
   } else if (kind == PH_DOWN) {
     g.epi = EPI_RESID;
     g.n_tiles = a.D / 128;
-    g.k_chunks = a.F / 64;
-    g.mw = lm + M_WDOWN;
-    g.mx = gm + G_ACT + a.mt_idx;
+    g.k_chunks = a.F / 128;
+    g.mw = lm + M_WDOWN3;
+    g.mx = gm + G_ACT3 + a.mt_idx;
   } else {  // PH_LM
     g.epi = EPI_ARGMAX;
     g.n_tiles = a.V / 128;
-    g.k_chunks = a.D / 64;
-    g.mw = gm + G_LM;
-    g.mx = gm + G_XN + a.mt_idx;
+    g.k_chunks = a.D / 128;
+    g.mw = gm + G_LM3;
+    g.mx = gm + G_XN3 + a.mt_idx;
   }
   g.units = (long long)g.n_tiles * g.k_chunks;
   return g;
@@ -742,14 +765,30 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           if (lane == 0) mbar_arrive(&acce[buf]);
           int n_contrib = 0;
           for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += ust_s[cc + 1] > ust_s[cc];
+          // The tile's head owner c_lo (it holds the first k unit) finishes the tile: the
+          // other contributors release a count after storing their partial, c_lo waits
+          // for all of them. A CTA is head owner of at most one split tile, so no CTA
+          // runs two fixups in a row (with a last-arriver rule all contributors finish
+          // together and one CTA can end up with both of its tiles). Waits point only to
+          // higher-indexed CTAs, whose parts are stored before they wait on anything.
           named_bar_sync(1, 128);
-          bool last = false;
           if (et == 0) tl_mark(a, n_ph, p, TL_S_PART);
-          if (et == 0) last = atom_add_acq_rel_gpu(a.tile_cnt + t, 1) == n_contrib - 1;
+          bool last = false;
+          if (c != c_lo) {
+            if (et == 0) red_release_gpu_add(a.tile_cnt + t, 1);
+          } else if (et == 0) {
+            const int code = wait_count_code(a.tile_cnt + t, n_contrib - 1, a.status);
+            fwd_diag(a, code, 17, p, it, t, n_contrib, *(volatile int*)(a.tile_cnt + t));
+            last = code == 1;
+            if (last) a.tile_cnt[t] = 0;
+          }
           if (et == 0) tl_mark(a, n_ph, p, TL_S_CNT);
           last = bcast(last);
+          if (c == c_lo && !last) {
+            ok = false;
+            break;
+          }
           if (last) {
-            if (et == 0) a.tile_cnt[t] = 0;
             for (int m0 = 0; m0 < a.Mt; m0 += 32) {
               const int n4 = min(32, a.Mt - m0) / 4;
 #pragma unroll
@@ -992,8 +1031,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   constexpr int d = D_HEAD;
   constexpr int halves = d / 64;
   const int S = a.stages;
-  const uint32_t x_bytes = (uint32_t)a.Mt * 128u;
-  const uint32_t stage_bytes = 16384u + x_bytes;
+  const uint32_t x_bytes = (uint32_t)a.Mt * 256u;  // two k chunks of Mt rows
+  const uint32_t stage_bytes = 32768u + x_bytes;
   uint8_t* sQ = smem + (size_t)S * stage_bytes;   // attention Q tile, d/64 blocks of 128 rows x 64
   uint8_t* scr = sQ + (size_t)128 * d * 2;         // P tile / epilogue staging
   unsigned long long* red = (unsigned long long*)(scr + kScratchBytes);
@@ -1128,9 +1167,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 ok = false;
                 break;
               }
-              mbar_arrive_expect_tx(&full[s], 16384u);
-              if (gp.gu) tma_load_3d_hint(st, gp.mw, &full[s], k * 64, t * 64, 0, pol_w);  // 64 gate + 64 up rows
-              else tma_load_2d_hint(st, gp.mw, &full[s], k * 64, t * 128, pol_w);
+              mbar_arrive_expect_tx(&full[s], 32768u);
+              if (gp.gu) tma_load_4d_hint(st, gp.mw, &full[s], 0, t * 64, 0, 2 * k, pol_w);  // gate + up rows
+              else tma_load_3d_hint(st, gp.mw, &full[s], 0, t * 128, 2 * k, pol_w);
             } else {
               if (!dep_ready(dep)) {
                 ok = false;
@@ -1138,7 +1177,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               }
               if (u == u0) tl_mark(a, n_ph, p, TL_X0);
               mbar_arrive_expect_tx(&full[s], x_bytes);
-              tma_load_2d(st + 16384, gp.mx, &full[s], k * 64, 0);
+              tma_load_3d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k);
             }
             last_ph[s] = (int)ph;
           }
@@ -1239,11 +1278,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               if (u == u0) tl_mark(a, n_ph, p, TL_M0);
               tc_fence_after();
               const uint32_t wa = smem_u32(stage_ptr(s));
-              const uint32_t xa = wa + 16384;
+              const uint32_t xa = wa + 32768;
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(d_tmem, sw128_desc(wa + kk * 32, 16, 1024), sw128_desc(xa + kk * 32, 16, 1024), idesc_g,
-                            (u > seg_start || kk > 0) ? 1u : 0u);
+              for (int c2 = 0; c2 < 2; ++c2) {  // the two 64-wide k chunks of the unit
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ss(d_tmem, sw128_desc(wa + c2 * 16384 + kk * 32, 16, 1024),
+                              sw128_desc(xa + c2 * (uint32_t)a.Mt * 128u + kk * 32, 16, 1024), idesc_g,
+                              (u > seg_start || c2 > 0 || kk > 0) ? 1u : 0u);
+              }
               mma_commit(&empty[s]);
             }
             if (!ok) break;

@@ -67,6 +67,32 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint6
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 map of rank 3 or 4 with explicit strides (bytes, dims 1..rank-1) and box.
+bool map_nd(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+            const uint32_t* box) {
+  EncodeTiledFn f = encode_fn();
+  if (!f || !base || rank < 3 || rank > 4) return false;
+  cuuint64_t d[4], st[3];
+  cuuint32_t b[4], es[4] = {1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) st[i] = strides[i];
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, st, b, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D view of a row-major [rows][cols] bf16 matrix as (64 columns, rows, cols/64 chunks) with
+// strides (row, 128 B): a box of (64, box_rows, 2) is two consecutive 64-wide k chunks.
+bool map_kpair(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[3] = {64, rows, cols / 64};
+  const uint64_t strides[2] = {cols * 2, 128};
+  const uint32_t box[3] = {64, box_rows, 2};
+  return map_nd(m, base, 3, dims, strides, box);
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int round_up(int x, int a) { return (x + a - 1) / a * a; }
 int next_pow2(int x) {
@@ -417,9 +443,10 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.Mt = round_up(a.M, 16);
   a.mt_idx = a.Mt / 16 - 1;
   const size_t stage = fwd_stage_bytes(a.Mt);
-  // 6 stages (about 96 KB of weight tiles in flight per SM) measured fastest; deeper
-  // rings put more requests in flight than HBM serves efficiently
-  a.stages = (int)std::min<size_t>(6, (kSmemLimit - fwd_fixed_smem(a.d)) / stage);
+  // 3-4 stages of 32 KB weight boxes (96-128 KB in flight per SM): a bare TMA stream of
+  // such boxes measured fastest at 4; deeper rings put more requests in flight than HBM
+  // serves efficiently
+  a.stages = (int)std::min<size_t>(4, (kSmemLimit - fwd_fixed_smem(a.d)) / stage);
   a.stages = std::max(2, std::min(a.stages, env_int("ORTHRUS_STAGES", a.stages)));
   const size_t smem = fwd_fixed_smem(a.d) + (size_t)a.stages * stage;
   a.cap = P->cap;
@@ -427,7 +454,7 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.batch = P->B;
   const int sms = num_sms();
   a.ck = P->fwd_ck;
-  a.lookahead = std::max(0, env_int("ORTHRUS_LOOKAHEAD", a.stages));
+  a.lookahead = std::max(0, env_int("ORTHRUS_LOOKAHEAD", 2));  // 2 k-pair tiles measured best
   a.pending = pending;
   a.draft_ids = draft;
   a.len = P->len;
@@ -771,7 +798,17 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
     ok = ok && map2d(P->lmap_mut(l, M_WDOWN), lp.w_down, F, D, 64, 128);
     ok = ok && map2d(P->lmap_mut(l, M_WDQKV), lp.wd_qkv, D, qkv_rows, 64, 128);
     ok = ok && map2d(P->lmap_mut(l, M_WDO), lp.wd_o, H * d, D, 64, 128);
-    ok = ok && map3d(P->lmap_mut(l, M_WGU3), lp.w_gu, D, F, 2, 64, 2);
+    ok = ok && map_kpair(P->lmap_mut(l, M_WQKV3), lp.w_qkv, D, qkv_rows, 128);
+    ok = ok && map_kpair(P->lmap_mut(l, M_WO3), lp.w_o, H * d, D, 128);
+    ok = ok && map_kpair(P->lmap_mut(l, M_WDOWN3), lp.w_down, F, D, 128);
+    ok = ok && map_kpair(P->lmap_mut(l, M_WDQKV3), lp.wd_qkv, D, qkv_rows, 128);
+    ok = ok && map_kpair(P->lmap_mut(l, M_WDO3), lp.wd_o, H * d, D, 128);
+    {  // (64 columns, d_ff rows, gate|up half, k chunk)
+      const uint64_t dims[4] = {64, (uint64_t)F, 2, (uint64_t)D / 64};
+      const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)F * D * 2, 128};
+      const uint32_t box[4] = {64, 64, 2, 2};
+      ok = ok && map_nd(P->lmap_mut(l, M_WGU4), lp.w_gu, 4, dims, strides, box);
+    }
     LayerNorms& ln = P->norms_host()[l];
     ln.attn_norm = lp.attn_norm;
     ln.mlp_norm = lp.mlp_norm;
@@ -781,11 +818,15 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
     ln.wd_k_norm = lp.wd_k_norm;
   }
   ok = ok && map2d(P->gmap_mut(G_LM), w->lm_head, D, V, 64, 128);
+  ok = ok && map_kpair(P->gmap_mut(G_LM3), w->lm_head, D, V, 128);
   const int rows = act_rows(max_rows);
   for (int i = 0; i < 8; ++i) {
     ok = ok && map2d(P->gmap_mut(G_XN + i), P->xn, D, rows, 64, 16 * (i + 1));
     ok = ok && map2d(P->gmap_mut(G_ATTN + i), P->attn, H * d, rows, 64, 16 * (i + 1));
     ok = ok && map2d(P->gmap_mut(G_ACT + i), P->act, F, rows, 64, 16 * (i + 1));
+    ok = ok && map_kpair(P->gmap_mut(G_XN3 + i), P->xn, D, rows, 16 * (i + 1));
+    ok = ok && map_kpair(P->gmap_mut(G_ATTN3 + i), P->attn, H * d, rows, 16 * (i + 1));
+    ok = ok && map_kpair(P->gmap_mut(G_ACT3 + i), P->act, F, rows, 16 * (i + 1));
   }
   ok = ok && map2d(P->gmap_mut(G_Q), P->qbuf, d, (uint64_t)rows * H + 128, 64, 128);
   const uint64_t zc = (uint64_t)L * P->B * Hkv;

@@ -60,7 +60,7 @@ def summarize(raw, L, sms, weight_bytes):
         if np.any(~np.isnan(col)):
             ends[p] = np.nanmax(col)
     rows = {}
-    prev = ends[0]
+    prev = ends[0] if not np.isnan(ends[0]) else np.nanmin(t)
     for p in range(1, nph):
         if np.isnan(ends[p]):
             continue
