@@ -740,8 +740,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           };
           const int c_lo = owner(t * kc), c_hi = owner((t + 1) * kc - 1);
           const bool add_h = gp.epi == EPI_RESID && c == c_hi;
+          // partial slot layout [token m / 4][weight row][m % 4]: a thread moves float4s and a
+          // warp's access is 512 contiguous bytes
           const int slot = 2 * c + (t == first_tile ? 0 : 1);
-          float* part = a.partial + (size_t)slot * (128 * 128) + (size_t)row * a.Mt;
+          float4* part = reinterpret_cast<float4*>(a.partial + (size_t)slot * (128 * 128)) + row;
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
             if (add_h) {
@@ -752,13 +754,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] += hv[j];
             }
-            const int n4 = min(32, a.Mt - m0) / 4;
             // partials stay in L2 (evict_last) while the weight stream passes through it
 #pragma unroll
-            for (int qq = 0; qq < 8; ++qq)
-              if (qq < n4)
-                st_f4_hint(reinterpret_cast<float4*>(part + m0) + qq,
-                           make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]), pol_keep);
+            for (int q4 = 0; q4 < 8; ++q4)
+              if (m0 + 4 * q4 < a.Mt)
+                st_f4_hint(part + (size_t)((m0 >> 2) + q4) * 128,
+                           make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]), pol_keep);
           }
           tc_fence_before();
           __syncwarp();
@@ -790,7 +791,6 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           }
           if (last) {
             for (int m0 = 0; m0 < a.Mt; m0 += 32) {
-              const int n4 = min(32, a.Mt - m0) / 4;
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = 0.f;
               int cc = c_lo;
@@ -811,23 +811,23 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                   const int sl = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
-                  const float4* pp = reinterpret_cast<const float4*>(
-                      a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128) + (size_t)row * a.Mt + m0);
+                  const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
+                                     (size_t)(m0 >> 2) * 128 + row;
 #pragma unroll
-                  for (int qq = 0; qq < 8; ++qq)
-                    x[q][qq] = (sl >= 0 && qq < n4) ? ld_f4_hint(pp + qq, pol_drop) : make_float4(0.f, 0.f, 0.f, 0.f);
+                  for (int q4 = 0; q4 < 8; ++q4)
+                    x[q][q4] = (sl >= 0 && m0 + 4 * q4 < a.Mt) ? ld_f4_hint(pp + (size_t)q4 * 128, pol_drop)
+                                                               : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
                 if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {  // fixed k order within and across rounds
+                for (int q = 0; q < 4; ++q)  // fixed k order within and across rounds
 #pragma unroll
-                  for (int qq = 0; qq < 8; ++qq) {
-                    v[4 * qq] += x[q][qq].x;
-                    v[4 * qq + 1] += x[q][qq].y;
-                    v[4 * qq + 2] += x[q][qq].z;
-                    v[4 * qq + 3] += x[q][qq].w;
+                  for (int q4 = 0; q4 < 8; ++q4) {
+                    v[4 * q4] += x[q][q4].x;
+                    v[4 * q4 + 1] += x[q][q4].y;
+                    v[4 * q4 + 2] += x[q][q4].z;
+                    v[4 * q4 + 3] += x[q][q4].w;
                   }
-                }
               }
               fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
             }

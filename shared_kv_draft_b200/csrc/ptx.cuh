@@ -167,6 +167,16 @@ __device__ __forceinline__ float4 ld_f4_hint(const float4* p, uint64_t policy) {
   return v;
 }
 
+__device__ __forceinline__ void st_f1_hint(float* p, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
+}
+
+__device__ __forceinline__ float ld_f1_hint(const float* p, uint64_t policy) {
+  float v;
+  asm volatile("ld.global.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(p), "l"(policy) : "memory");
+  return v;
+}
+
 // generic-proxy global writes <-> later async-proxy (TMA) accesses
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
