@@ -108,6 +108,7 @@ struct FwdArgs {
   int view;                  // VIEW_DRAFT / VIEW_VERIFY
   int nb, Q, M, Mt, mt_idx, stages, cap, max_block, batch;
   int lookahead;             // weight tiles the weight producer loads ahead of a phase's input dependency
+  int poll_ns;               // sleep between polls of a phase counter
   int ck;                    // keys per attention chunk: fixed per plan (multiple of 64, >= capacity / 16),
                              // so a row's softmax runs over the same absolute key chunks whatever
                              // the block size: verify rows equal the plain AR rows bit for bit
@@ -564,7 +565,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
     bool r = false;
     if (et == 0) {
       const int tgt = phase_target(a, g, dep);
-      const int code = wait_count_code(a.phase_cnt + dep, tgt, a.status);
+      const int code = wait_count_code(a.phase_cnt + dep, tgt, a.status, a.poll_ns);
       fwd_diag(a, code, 12, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
       r = code == 1;
     }
@@ -869,6 +870,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             ok = false;
             break;
           }
+          if (et == 0) tl_mark(a, n_ph, p, j == 0 ? TL_R0 : TL_S_ACC);  // score tile ready
           tc_fence_after();
           const int key0 = t.key_lo + j * 64;
           float mx = -INFINITY;
@@ -881,7 +883,8 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               if (key0 + c0 + tt < lim) mx = fmaxf(mx, v[tt] * a.scale_log2);
           }
           const float m_new = fmaxf(m_run, mx);
-          const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
+          const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_PART);  // row maxima done
           float sum = 0.f;
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -890,8 +893,8 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             uint32_t pk[16];
 #pragma unroll
             for (int tt = 0; tt < 32; tt += 2) {
-              const float p0 = (key0 + c0 + tt < lim) ? exp2f(v[tt] * a.scale_log2 - m_new) : 0.f;
-              const float p1 = (key0 + c0 + tt + 1 < lim) ? exp2f(v[tt + 1] * a.scale_log2 - m_new) : 0.f;
+              const float p0 = (key0 + c0 + tt < lim) ? fast_exp2(v[tt] * a.scale_log2 - m_new) : 0.f;
+              const float p1 = (key0 + c0 + tt + 1 < lim) ? fast_exp2(v[tt + 1] * a.scale_log2 - m_new) : 0.f;
               sum += p0 + p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
               pk[tt / 2] = *reinterpret_cast<uint32_t*>(&h2);
@@ -922,10 +925,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(p_full);
+          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_CNT);  // P written
           if (!bar_wait_all(o_full, (uint32_t)ta & 1u, 15)) {
             ok = false;
             break;
           }
+          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);  // P V done
           tc_fence_after();
 #pragma unroll
           for (int c0 = 0; c0 < d; c0 += 32) {
@@ -938,8 +943,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(t_done);
+          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_EPI);  // O accumulated
         }
         if (!ok) break;
+        if (et == 0) tl_mark(a, n_ph, p, TL_R1);
         const int H = a.H;
         if (t.n_chunks == 1) {
           if (row_ok) {
@@ -955,10 +962,11 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             }
           }
         } else {
+          // partial O in a [chunk][d/4][row][4] layout: a warp's float4 stores are 512 contiguous bytes
           const size_t pidx = ((size_t)t.slot * kMaxChunks + t.chunk) * 128 + row;
-          float* po = a.att_o + pidx * d;
+          float4* po = reinterpret_cast<float4*>(a.att_o) + ((size_t)t.slot * kMaxChunks + t.chunk) * (d / 4) * 128 + row;
 #pragma unroll
-          for (int e = 0; e < d; e += 4) __stcg(reinterpret_cast<float4*>(po + e), make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
+          for (int e = 0; e < d; e += 4) __stcg(po + (size_t)(e / 4) * 128, make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
           __stcg(a.att_ml + pidx, make_float2(m_run, l_run));
         }
         signal(p);
@@ -972,12 +980,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         break;
       }
       if (et == 0) tl_mark(a, n_ph, p, TL_E0);
-      constexpr int per = d / 8;  // columns per thread
+      constexpr int per = d / 8;  // columns per thread: thread et takes row et % 16 and column block et / 16
       for (int u = c; u < g.comb_units; u += Gd) {
         const int slot = u / (128 / kCombineRows), grp = u % (128 / kCombineRows);
         const int nch = slot_pre[slot + 1] - slot_pre[slot];
         const int r_t = slot % g.rt, kvh = (slot / g.rt) % a.Hkv, bb = slot / (g.rt * a.Hkv);
-        const int r = grp * kCombineRows + (et >> 3), sub = et & 7;
+        const int r = grp * kCombineRows + (et & 15), sub = et >> 4;
         const int grow = r_t * 128 + r;
         if (nch > 1 && grow < g.rows_per_slot) {
           const int i = grow / a.G, gg = grow - i * a.G;
@@ -990,13 +998,13 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           for (int e = 0; e < per; ++e) acc[e] = 0.f;
           for (int ch = 0; ch < nch; ++ch) {
             const float2 v = __ldcg(ml + ch * 128);
-            const float w = (v.x == -INFINITY) ? 0.f : exp2f(v.x - mstar);
+            const float w = (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - mstar);
             L += v.y * w;
-            const float4* po = reinterpret_cast<const float4*>(
-                a.att_o + (((size_t)slot * kMaxChunks + ch) * 128 + r) * d + sub * per);
+            const float4* po = reinterpret_cast<const float4*>(a.att_o) +
+                               (((size_t)slot * kMaxChunks + ch) * (d / 4) + sub * (per / 4)) * 128 + r;
 #pragma unroll
             for (int e = 0; e < per / 4; ++e) {
-              const float4 x = __ldcg(po + e);
+              const float4 x = __ldcg(po + (size_t)e * 128);
               acc[4 * e] += w * x.x;
               acc[4 * e + 1] += w * x.y;
               acc[4 * e + 2] += w * x.z;
@@ -1129,7 +1137,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
       auto dep_ready = [&](int dep) -> bool {
         if (dep <= known_done) return true;
         const int tgt = phase_target(a, g, dep);
-        const int r = wait_count_code(a.phase_cnt + dep, tgt, a.status);
+        const int r = wait_count_code(a.phase_cnt + dep, tgt, a.status, a.poll_ns);
         if (r != 1) {
           fwd_diag(a, r, 3, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
           return false;
@@ -1188,17 +1196,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
             const int zc = (l * a.batch + t.bb) * a.Hkv + t.kvh;
             const int qrow = (t.bb * a.Hkv + t.kvh) * g.rows_per_slot + t.r * 128;
             const int n_loads = 2 * t.tiles;
-            if (!wprod) {  // Q tile into its own region once the previous unit's S MMAs are done
+            // Cache keys below len were written by earlier launches: their K/V tiles are
+            // loaded without waiting for this layer's q/k/v phase. The Q tile and block
+            // keys wait for it; Q goes out before the first such load, or after the first
+            // K/V pair when that pair is independent.
+            bool q_issued = false;
+            auto issue_q = [&]() -> bool {
+              if (!dep_ready(dep)) return false;
+              mbar_arrive_expect_tx(q_full, 16384u * halves);
+              for (int hh = 0; hh < halves; ++hh) tma_load_2d(sQ + hh * 16384, gm + G_Q, q_full, hh * 64, qrow);
+              q_issued = true;
+              return true;
+            };
+            auto independent = [&](int key0) { return !t.blk && key0 + 64 <= t.n; };
+            if (!wprod) {  // Q region free once the previous unit's S MMAs are done
               const int r = mbar_wait_code(q_empty, ((uint32_t)qu & 1u) ^ 1u, a.status);
               if (r != 1) fwd_diag(a, r, 4, p, it, qu);
-              if (r != 1 || !dep_ready(dep)) {
+              if (r != 1 || (!independent(t.key_lo) && !issue_q())) {
                 ok = false;
                 break;
               }
-              mbar_arrive_expect_tx(q_full, 16384u * halves);
-              for (int hh = 0; hh < halves; ++hh) tma_load_2d(sQ + hh * 16384, gm + G_Q, q_full, hh * 64, qrow);
             }
             for (int j = 0; j < n_loads; ++j, ++it) {
+              const int key0 = t.key_lo + (j >> 1) * 64;
+              // Q before any wait that needs this unit's own S MMAs (with two ring stages
+              // the stage of load j = 2 is that of load 0)
+              if (!wprod && (j >= 2 || !independent(key0)) && !q_issued && !issue_q()) {
+                ok = false;
+                break;
+              }
               const int s = it % S;
               const uint32_t ph = (uint32_t)(it / S) & 1u;
               const int r = mbar_wait_code(&empty[s], ph ^ 1u, a.status);
@@ -1212,16 +1238,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 mbar_arrive(&full[s]);  // attention tiles all come from the activation producer
                 continue;
               }
-              if (!dep_ready(dep)) {
+              if (!independent(key0) && !dep_ready(dep)) {
                 ok = false;
                 break;
               }
               uint8_t* st = stage_ptr(s);
-              const int key0 = t.key_lo + (j >> 1) * 64;
               const bool is_v = j & 1;
               const CUtensorMap* mp = t.blk ? (is_v ? gm + G_VB64 : gm + G_KB64) : (is_v ? gm + G_VC64 : gm + G_KC64);
               mbar_arrive_expect_tx(&full[s], 8192u * halves);
               for (int hh = 0; hh < halves; ++hh) tma_load_3d(st + hh * 8192, mp, &full[s], hh * 64, key0, zc);
+            }
+            if (ok && !wprod && !q_issued && !issue_q()) {
+              ok = false;
+              break;
             }
           }
         }

@@ -455,6 +455,7 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   const int sms = num_sms();
   a.ck = P->fwd_ck;
   a.lookahead = std::max(0, env_int("ORTHRUS_LOOKAHEAD", 2));  // 2 k-pair tiles measured best
+  a.poll_ns = std::max(0, env_int("ORTHRUS_POLL_NS", 64));
   a.pending = pending;
   a.draft_ids = draft;
   a.len = P->len;

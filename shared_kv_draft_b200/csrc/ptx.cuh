@@ -187,12 +187,12 @@ __device__ __forceinline__ void sleep_ns(uint32_t ns) { asm volatile("nanosleep.
 // Wait until *cnt >= target (acquire). False once the status word holds an
 // error or after about 2 s (then ORTHRUS_ERR_TIMEOUT is recorded).
 // 1 = reached, 0 = gave up because the status word holds an error, -1 = timed out here.
-__device__ __forceinline__ int wait_count_code(const int* cnt, int target, int* status) {
+__device__ __forceinline__ int wait_count_code(const int* cnt, int target, int* status, uint32_t poll_ns = 64) {
   if (ld_acquire_gpu(cnt) >= target) return 1;
   const long long t0 = clock64();
 #pragma unroll 1
   for (uint32_t it = 0;; ++it) {
-    sleep_ns(64);
+    sleep_ns(poll_ns);
     if (ld_acquire_gpu(cnt) >= target) return 1;
     if ((it & 255u) == 0u) {
       if (*(volatile int*)status != 0) return 0;
@@ -374,6 +374,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz.f32, a few ulp): used for
+// softmax weights, which are rounded to bf16 right after.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
