@@ -745,7 +745,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           // warp's access is 512 contiguous bytes
           const int slot = 2 * c + (t == first_tile ? 0 : 1);
           float4* part = reinterpret_cast<float4*>(a.partial + (size_t)slot * (128 * 128)) + row;
-          for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+          // the head owner keeps its own part in TMEM (re-read after the others arrive)
+          const bool head = c == c_lo;
+          for (int m0 = 0; !head && m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
             if (add_h) {
               float hv[32];
@@ -762,9 +764,11 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                 st_f4_hint(part + (size_t)((m0 >> 2) + q4) * 128,
                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]), pol_keep);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acce[buf]);
+          if (!head) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[buf]);
+          }
           int n_contrib = 0;
           for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += ust_s[cc + 1] > ust_s[cc];
           // The tile's head owner c_lo (it holds the first k unit) finishes the tile: the
@@ -792,9 +796,8 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           }
           if (last) {
             for (int m0 = 0; m0 < a.Mt; m0 += 32) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = 0.f;
-              int cc = c_lo;
+              tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
+              int cc = c_lo + 1;
               while (cc <= c_hi) {
                 // up to four contributors per round, their loads all in flight together
                 int s0 = -1, s1 = -1, s2 = -1, s3 = -1;
@@ -832,6 +835,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               }
               fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[buf]);
             if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
             signal(p);
             if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
