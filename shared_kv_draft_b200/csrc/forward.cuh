@@ -760,7 +760,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             // partials stay in L2 (evict_last) while the weight stream passes through it
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
-              if (m0 + 4 * q4 < a.Mt)
+              if (m0 + 4 * q4 < m_valid)  // only token columns that exist
                 st_f4_hint(part + (size_t)((m0 >> 2) + q4) * 128,
                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]), pol_keep);
           }
@@ -819,7 +819,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                                      (size_t)(m0 >> 2) * 128 + row;
 #pragma unroll
                   for (int q4 = 0; q4 < 8; ++q4)
-                    x[q][q4] = (sl >= 0 && m0 + 4 * q4 < a.Mt) ? ld_f4_hint(pp + (size_t)q4 * 128, pol_drop)
+                    x[q][q4] = (sl >= 0 && m0 + 4 * q4 < m_valid) ? ld_f4_hint(pp + (size_t)q4 * 128, pol_drop)
                                                                : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
                 if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);

@@ -111,18 +111,31 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t pari
   }
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes
+// or about `ns` nanoseconds pass, instead of spinning and taking issue slots from
+// the other warp on its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Same as mbar_wait_abortable, but tells the two failures apart: 1 = phase
 // completed, 0 = gave up because the status word already held an error,
 // -1 = this wait ran out of time (ORTHRUS_ERR_TIMEOUT recorded).
 __device__ __forceinline__ int mbar_wait_code(uint64_t* bar, uint32_t parity, int* status) {
-#pragma unroll 1
-  for (int i = 0; i < 4096; ++i)
-    if (mbar_try_wait(bar, parity)) return 1;
+  if (mbar_try_wait(bar, parity)) return 1;
   const long long t0 = clock64();
 #pragma unroll 1
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return 1;
-    if ((it & 1023u) == 0u) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return 1;
+    if ((it & 15u) == 0u) {
       if (*(volatile int*)status != 0) return 0;
       if (clock64() - t0 > kWaitLimitCycles) {
         set_status(status, ORTHRUS_ERR_TIMEOUT);
