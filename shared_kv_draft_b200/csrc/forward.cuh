@@ -532,7 +532,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                                                   unsigned long long* red, float* rstd_s, const int* lens_s,
                                                   const int* slot_pre, int* ust_s, uint64_t* accf, uint64_t* acce,
                                                   uint64_t* full, uint64_t* s_full, uint64_t* p_full,
-                                                  uint64_t* o_full, uint64_t* t_done, int* flag,
+                                                  uint64_t* o_full, int* flag,
                                                   uint32_t tmem_base, uint32_t tS, uint32_t tO) {
   constexpr int d = D_HEAD;
   constexpr int halves = d / 64;
@@ -867,9 +867,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           kv_end = min(t.n + i_max + 1, t.key_hi);
         }
         if (!row_ok) lim = t.key_lo;
-        float o[d];
-#pragma unroll
-        for (int e = 0; e < d; ++e) o[e] = 0.f;
+        // O accumulates in TMEM across the unit's key tiles (P V MMAs with accumulate);
+        // when a row's running maximum moves, the row of O is rescaled in TMEM before
+        // the next P V. O is read into registers once, after the last tile.
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; j < t.tiles; ++j, it += 2, ++ta) {
           if (!bar_wait_all(s_full, (uint32_t)ta & 1u, 14)) {
@@ -879,28 +879,42 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           if (et == 0) tl_mark(a, n_ph, p, j == 0 ? TL_R0 : TL_S_ACC);  // score tile ready
           tc_fence_after();
           const int key0 = t.key_lo + j * 64;
+          float sv[64];
+          tmem_ld32(tS + lane_base, sv);
+          tmem_ld32(tS + lane_base + 32, sv + 32);
           float mx = -INFINITY;
 #pragma unroll
-          for (int c0 = 0; c0 < 64; c0 += 32) {
-            float v[32];
-            tmem_ld32(tS + lane_base + c0, v);
-#pragma unroll
-            for (int tt = 0; tt < 32; ++tt)
-              if (key0 + c0 + tt < lim) mx = fmaxf(mx, v[tt] * a.scale_log2);
-          }
+          for (int tt = 0; tt < 64; ++tt)
+            if (key0 + tt < lim) mx = fmaxf(mx, sv[tt] * a.scale_log2);
           const float m_new = fmaxf(m_run, mx);
           const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
           if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_PART);  // row maxima done
+          if (j > 0) {
+            // the previous tile's P V must be complete before O is rescaled
+            if (!bar_wait_all(o_full, (uint32_t)(ta - 1) & 1u, 15)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st are per warp
+#pragma unroll
+              for (int c0 = 0; c0 < d; c0 += 32) {
+                float v[32];
+                tmem_ld32(tO + lane_base + c0, v);
+#pragma unroll
+                for (int tt = 0; tt < 32; ++tt) v[tt] *= alpha;
+                tmem_st32(tO + lane_base + c0, v);
+              }
+            }
+          }
           float sum = 0.f;
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 32) {
-            float v[32];
-            tmem_ld32(tS + lane_base + c0, v);
             uint32_t pk[16];
 #pragma unroll
             for (int tt = 0; tt < 32; tt += 2) {
-              const float p0 = (key0 + c0 + tt < lim) ? fast_exp2(v[tt] * a.scale_log2 - m_new) : 0.f;
-              const float p1 = (key0 + c0 + tt + 1 < lim) ? fast_exp2(v[tt + 1] * a.scale_log2 - m_new) : 0.f;
+              const float p0 = (key0 + c0 + tt < lim) ? fast_exp2(sv[c0 + tt] * a.scale_log2 - m_new) : 0.f;
+              const float p1 = (key0 + c0 + tt + 1 < lim) ? fast_exp2(sv[c0 + tt + 1] * a.scale_log2 - m_new) : 0.f;
               sum += p0 + p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
               pk[tt / 2] = *reinterpret_cast<uint32_t*>(&h2);
@@ -914,6 +928,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             }
           }
           l_run = l_run * alpha + sum;
+          m_run = m_new;
           // V rows of keys no row may see are zeroed (stale or poisoned cache rows)
           if (key0 + 64 > kv_end && row < 64 && key0 + row >= kv_end) {
             const int vs = (it + 1) % S;
@@ -932,26 +947,18 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           __syncwarp();
           if (lane == 0) mbar_arrive(p_full);
           if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_CNT);  // P written
-          if (!bar_wait_all(o_full, (uint32_t)ta & 1u, 15)) {
-            ok = false;
-            break;
-          }
-          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);  // P V done
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < d; c0 += 32) {
-            float v[32];
-            tmem_ld32(tO + lane_base + c0, v);
-#pragma unroll
-            for (int tt = 0; tt < 32; ++tt) o[c0 + tt] = o[c0 + tt] * alpha + v[tt];
-          }
-          m_run = m_new;
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(t_done);
-          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_EPI);  // O accumulated
         }
         if (!ok) break;
+        // the unit's last P V, then O into registers
+        if (!bar_wait_all(o_full, (uint32_t)(ta - 1) & 1u, 15)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float o[d];
+#pragma unroll
+        for (int c0 = 0; c0 < d; c0 += 32) tmem_ld32(tO + lane_base + c0, o + c0);
+        tc_fence_before();
         if (et == 0) tl_mark(a, n_ph, p, TL_R1);
         const int H = a.H;
         if (t.n_chunks == 1) {
@@ -1062,7 +1069,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   uint64_t* s_full = acce + 2;
   uint64_t* p_full = s_full + 1;
   uint64_t* o_full = s_full + 2;
-  uint64_t* t_done = s_full + 3;
   uint64_t* done = s_full + 4;
   uint64_t* q_full = s_full + 5;
   uint64_t* q_empty = s_full + 6;
@@ -1088,7 +1094,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
     mbar_init(s_full, 1);
     mbar_init(p_full, 4);
     mbar_init(o_full, 1);
-    mbar_init(t_done, 4);
     mbar_init(done, 1);
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
@@ -1356,15 +1361,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               mma_commit(s_full);
               mma_commit(&empty[ks]);
               if (j == t.tiles - 1) mma_commit(q_empty);  // last read of this unit's Q tile
+              // P of this tile written (and O rescaled) by the softmax warps, V landed
               r = mbar_wait_code(p_full, (uint32_t)ta & 1u, a.status);
               if (r == 1) {
                 r = mbar_wait_code(&full[vs], (uint32_t)((it + 1) / S) & 1u, a.status);
-                if (r == 1 && ta > 0) {
-                  r = mbar_wait_code(t_done, (uint32_t)(ta - 1) & 1u, a.status);
-                  if (r != 1) fwd_diag(a, r, 11, p, it, ta);
-                } else if (r != 1) {
-                  fwd_diag(a, r, 10, p, it, vs);
-                }
+                if (r != 1) fwd_diag(a, r, 10, p, it, vs);
               } else {
                 fwd_diag(a, r, 9, p, it, ta);
               }
@@ -1377,7 +1378,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, 8192, 1024), idO,
-                            kk > 0 ? 1u : 0u);
+                            (j > 0 || kk > 0) ? 1u : 0u);
               mma_commit(o_full);
               mma_commit(&empty[vs]);
             }
@@ -1391,7 +1392,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   } else {
     // ======================= epilogue warps =======================
     fwd_epilogue_role<D_HEAD>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, ust_s, accf, acce, full,
-                              s_full, p_full, o_full, t_done, flag, tmem_base, tS, tO);
+                              s_full, p_full, o_full, flag, tmem_base, tS, tO);
   }
 
   // ---------------- teardown ----------------
