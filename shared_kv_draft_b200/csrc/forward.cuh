@@ -699,6 +699,56 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         gam = l + 1 < a.L ? a.norms[l + 1].attn_norm : a.final_norm;
       }
       const int first_tile = (int)(u0 / kc);
+      const int m_valid = min(a.Mt, a.M);
+      // owner of unit uu = the CTA whose non-empty range holds it (largest c with start <= uu)
+      auto owner = [&](int uu) {
+        int lo = 0, hi = Gd - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (ust_s[mid] <= uu) lo = mid;
+          else hi = mid - 1;
+        }
+        return lo;
+      };
+      // partial slot of contributor cc to tile t: its first or its last segment
+      auto part_slot = [&](int cc, int t) { return 2 * cc + (ust_s[cc] / kc == t ? 0 : 1); };
+      // next (up to) four non-empty contributors from cc on, in k order
+      auto gather4 = [&](int& cc, int c_hi, int& s0, int& s1, int& s2, int& s3, int t) {
+        s0 = s1 = s2 = s3 = -1;
+        for (int q = 0; q < 4 && cc <= c_hi; ++cc) {
+          if (ust_s[cc + 1] > ust_s[cc]) {
+            const int sl = part_slot(cc, t);
+            if (q == 0) s0 = sl;
+            else if (q == 1) s1 = sl;
+            else if (q == 2) s2 = sl;
+            else s3 = sl;
+            ++q;
+          }
+        }
+      };
+      auto load4 = [&](float4 (&x)[4][8], int s0, int s1, int s2, int s3, int m0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int sl = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
+          const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
+                             (size_t)(m0 >> 2) * 128 + row;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            x[q][q4] = (sl >= 0 && m0 + 4 * q4 < m_valid) ? ld_f4_hint(pp + (size_t)q4 * 128, pol_drop)
+                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      };
+      auto add4 = [&](float* v, const float4 (&x)[4][8]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)  // fixed k order within and across rounds
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            v[4 * q4] += x[q][q4].x;
+            v[4 * q4 + 1] += x[q][q4].y;
+            v[4 * q4 + 2] += x[q][q4].z;
+            v[4 * q4 + 3] += x[q][q4].w;
+          }
+      };
       long long u = u0;
       while (ok && u < u1) {
         const int t = (int)(u / kc);
@@ -706,18 +756,17 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         u = seg_end;
         const int buf = seg & 1, use = seg >> 1;
         ++seg;
-        if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
-          ok = false;
-          break;
-        }
-        if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
-        tc_fence_after();
         const int nt = t;
-        const int m_valid = min(a.Mt, a.M);
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * 128;
         const bool whole = seg_start == (long long)t * kc && seg_end == (long long)(t + 1) * kc;
         float v[32];
         if (whole) {
+          if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
+            ok = false;
+            break;
+          }
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
+          tc_fence_after();
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
             fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
@@ -728,26 +777,28 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
           signal(p);
           if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
-        } else {
-          // owner of unit u = the CTA whose non-empty range holds it (largest c with start <= u)
-          auto owner = [&](int uu) {
-            int lo = 0, hi = Gd - 1;
-            while (lo < hi) {
-              const int mid = (lo + hi + 1) >> 1;
-              if (ust_s[mid] <= uu) lo = mid;
-              else hi = mid - 1;
-            }
-            return lo;
-          };
-          const int c_lo = owner(t * kc), c_hi = owner((t + 1) * kc - 1);
+          continue;
+        }
+        const int c_lo = owner(t * kc), c_hi = owner((t + 1) * kc - 1);
+        // The tile's head owner c_lo (it holds the first k unit) finishes the tile: the
+        // other contributors release a count after storing their partial, c_lo waits
+        // for all of them. A CTA is head owner of at most one split tile (its last
+        // segment), so no CTA runs two fixups in a row. Waits point only to higher-indexed
+        // CTAs, whose parts are stored (their first segment) before they wait on anything.
+        const bool head = c == c_lo;
+        if (!head) {
+          if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
+            ok = false;
+            break;
+          }
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
+          tc_fence_after();
           const bool add_h = gp.epi == EPI_RESID && c == c_hi;
           // partial slot layout [token m / 4][weight row][m % 4]: a thread moves float4s and a
           // warp's access is 512 contiguous bytes
           const int slot = 2 * c + (t == first_tile ? 0 : 1);
           float4* part = reinterpret_cast<float4*>(a.partial + (size_t)slot * (128 * 128)) + row;
-          // the head owner keeps its own part in TMEM (re-read after the others arrive)
-          const bool head = c == c_lo;
-          for (int m0 = 0; !head && m0 < a.Mt; m0 += 32) {
+          for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
             if (add_h) {
               float hv[32];
@@ -764,85 +815,63 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                 st_f4_hint(part + (size_t)((m0 >> 2) + q4) * 128,
                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]), pol_keep);
           }
-          if (!head) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce[buf]);
-          }
-          int n_contrib = 0;
-          for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += ust_s[cc + 1] > ust_s[cc];
-          // The tile's head owner c_lo (it holds the first k unit) finishes the tile: the
-          // other contributors release a count after storing their partial, c_lo waits
-          // for all of them. A CTA is head owner of at most one split tile, so no CTA
-          // runs two fixups in a row (with a last-arriver rule all contributors finish
-          // together and one CTA can end up with both of its tiles). Waits point only to
-          // higher-indexed CTAs, whose parts are stored before they wait on anything.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce[buf]);
           named_bar_sync(1, 128);
           if (et == 0) tl_mark(a, n_ph, p, TL_S_PART);
-          bool last = false;
-          if (c != c_lo) {
-            if (et == 0) red_release_gpu_add(a.tile_cnt + t, 1);
-          } else if (et == 0) {
-            const int code = wait_count_code(a.tile_cnt + t, n_contrib - 1, a.status);
-            fwd_diag(a, code, 17, p, it, t, n_contrib, *(volatile int*)(a.tile_cnt + t));
-            last = code == 1;
-            if (last) a.tile_cnt[t] = 0;
-          }
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_CNT);
-          last = bcast(last);
-          if (c == c_lo && !last) {
-            ok = false;
-            break;
-          }
-          if (last) {
-            for (int m0 = 0; m0 < a.Mt; m0 += 32) {
-              tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
-              int cc = c_lo + 1;
-              while (cc <= c_hi) {
-                // up to four contributors per round, their loads all in flight together
-                int s0 = -1, s1 = -1, s2 = -1, s3 = -1;
-                for (int q = 0; q < 4 && cc <= c_hi; ++cc) {
-                  if (ust_s[cc + 1] > ust_s[cc]) {
-                    const int sl = 2 * cc + (ust_s[cc] / kc == t ? 0 : 1);
-                    if (q == 0) s0 = sl;
-                    else if (q == 1) s1 = sl;
-                    else if (q == 2) s2 = sl;
-                    else s3 = sl;
-                    ++q;
-                  }
-                }
-                float4 x[4][8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const int sl = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
-                  const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
-                                     (size_t)(m0 >> 2) * 128 + row;
-#pragma unroll
-                  for (int q4 = 0; q4 < 8; ++q4)
-                    x[q][q4] = (sl >= 0 && m0 + 4 * q4 < m_valid) ? ld_f4_hint(pp + (size_t)q4 * 128, pol_drop)
-                                                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)  // fixed k order within and across rounds
-#pragma unroll
-                  for (int q4 = 0; q4 < 8; ++q4) {
-                    v[4 * q4] += x[q][q4].x;
-                    v[4 * q4 + 1] += x[q][q4].y;
-                    v[4 * q4 + 2] += x[q][q4].z;
-                    v[4 * q4 + 3] += x[q][q4].w;
-                  }
-              }
-              fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acce[buf]);
-            if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
-            signal(p);
-            if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
-          }
+          if (et == 0) red_release_gpu_add(a.tile_cnt + t, 1);
+          continue;
         }
+        // Head owner. The other contributors stored their parts at the start of their
+        // ranges, long before this CTA's own part (the end of its range) is accumulated:
+        // their count is awaited and their first token group loaded while the MMAs of
+        // the last k units still run.
+        int n_contrib = 0;
+        for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += ust_s[cc + 1] > ust_s[cc];
+        bool ready = false;
+        if (et == 0) {
+          const int code = wait_count_code(a.tile_cnt + t, n_contrib - 1, a.status);
+          fwd_diag(a, code, 17, p, it, t, n_contrib, *(volatile int*)(a.tile_cnt + t));
+          ready = code == 1;
+          if (ready) a.tile_cnt[t] = 0;
+        }
+        if (et == 0) tl_mark(a, n_ph, p, TL_S_CNT);
+        if (!bcast(ready)) {
+          ok = false;
+          break;
+        }
+        int cc0 = c_lo + 1, s0, s1, s2, s3;
+        gather4(cc0, c_hi, s0, s1, s2, s3, t);
+        float4 x[4][8];
+        load4(x, s0, s1, s2, s3, 0);
+        if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
+          ok = false;
+          break;
+        }
+        if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
+        tc_fence_after();
+        for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+          tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
+          int cc = c_lo + 1;
+          if (m0 == 0) {
+            add4(v, x);
+            cc = cc0;
+          }
+          while (cc <= c_hi) {
+            gather4(cc, c_hi, s0, s1, s2, s3, t);
+            load4(x, s0, s1, s2, s3, m0);
+            add4(v, x);
+          }
+          if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
+          fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[buf]);
+        if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
+        signal(p);
+        if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
       }
       it += (int)(u1 - u0);
       if (et == 0) tl_mark(a, n_ph, p, TL_E1);
