@@ -453,10 +453,63 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
   named_bar_sync(1, 128);
 }
 
+// SwiGLU epilogue of the gate/up projection on 32 token rows [m0, m0+32) of one
+// tile: rows 0..63 are the gate rows of features nt*64.., rows 64..127 the matching
+// up rows; act = silu(gate) * up in bf16.
+__device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
+                                                    int m_valid, float* epi) {
+  // stage the whole 128 x 32 group, then every thread takes one feature for 16 tokens
+  // (all four warps run the same code)
+#pragma unroll
+  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+  named_bar_sync(1, 128);
+  const int f = row & 63, j0 = (row >> 6) * 16;
+  __nv_bfloat16* dst = a.act + (size_t)(m0 + j0) * a.F + nt * 64 + f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (m0 + j0 + j < m_valid) {
+      const float g = epi[(j0 + j) * kEpiStride + f];
+      const float u = epi[(j0 + j) * kEpiStride + 64 + f];
+      // fast reciprocal: an IEEE divide has a slow-path branch per element that serialises the loop
+      dst[(size_t)j * a.F] = __float2bfloat16(__fdividef(g, 1.0f + __expf(-g)) * u);
+    }
+  }
+  named_bar_sync(1, 128);
+}
+
+// Greedy head of the LM projection on 32 token rows [m0, m0+32) of one 128-row
+// vocabulary tile: optional fp32 logits, NaN check, and the running argmax key of
+// each token row (max over the tile's rows, then one atomic per row).
+__device__ __forceinline__ void fwd_argmax_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
+                                                    int m_valid, unsigned long long* red) {
+  const int ew = (threadIdx.x >> 5) - 2, lane = threadIdx.x & 31;
+  const uint32_t col = nt * 128 + row;  // vocabulary index
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int m = m0 + j;
+    unsigned long long key = 0ull;
+    if (m < m_valid) {
+      if (a.logits) a.logits[(size_t)m * a.V + col] = v[j];
+      if (isnan(v[j])) set_status(a.status, ORTHRUS_ERR_NAN);
+      else key = argmax_key(v[j], col);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) key = ull_max(key, __shfl_xor_sync(0xffffffffu, key, o));
+    if (lane == 0) red[ew * 32 + j] = key;
+  }
+  named_bar_sync(1, 128);
+  if (ew == 0) {
+    const int m = m0 + lane;
+    const unsigned long long k = ull_max(ull_max(red[lane], red[32 + lane]), ull_max(red[64 + lane], red[96 + lane]));
+    if (m < m_valid && k != 0ull) atomicMax(a.amax + m, k);
+  }
+  named_bar_sync(1, 128);
+}
+
 // Epilogue of one 32-row group for the GEMM phase kinds. Consumers of a
 // normalised input first scale by rstd of the token row.
 template <int D_HEAD>
-__device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const GemmArgs& ga, const QkvCtx& qc, const int* lens_s,
+__device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const QkvCtx& qc, const int* lens_s,
                                              int epi_kind, float* v, int row, int m0, int nt, int m_valid, float* epi,
                                              unsigned long long* red, const float* rstd_s, const float* gam,
                                              bool h_in_v = false) {
@@ -467,8 +520,8 @@ __device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const GemmArgs& g
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] *= rstd_s[m0 + j];
   if (epi_kind == EPI_QKV) fwd_qkv_epilogue<D_HEAD>(a, qc, v, row, m0, nt, m_valid, epi, lens_s);
-  else if (epi_kind == EPI_SWIGLU) epilogue_group<EPI_SWIGLU>(ga, v, row, m0, 0, nt, m_valid, epi, red);
-  else epilogue_group<EPI_ARGMAX>(ga, v, row, m0, 0, nt, m_valid, epi, red);
+  else if (epi_kind == EPI_SWIGLU) fwd_swiglu_epilogue(a, v, row, m0, nt, m_valid, epi);
+  else fwd_argmax_epilogue(a, v, row, m0, nt, m_valid, red);
 }
 
 }  // namespace orthrus
@@ -658,16 +711,6 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         named_bar_sync(1, 128);
       }
-      GemmArgs ga;
-      memset(&ga, 0, sizeof(ga));
-      ga.M = a.M;
-      ga.Mt = a.Mt;
-      ga.status = a.status;
-      ga.out_bf16 = a.act;
-      ga.ld_out = a.F;
-      ga.amax = a.amax;
-      ga.logits = a.logits;
-      ga.ld_logits = a.V;
       const float* gam = nullptr;
       QkvCtx qc;
       qc.kdst = qc.vdst = nullptr;
@@ -769,7 +812,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_after();
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
-            fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
+            fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
           }
           tc_fence_before();
           __syncwarp();
@@ -864,7 +907,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             add4(v, x);
           }
           if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
-          fwd_epilogue<D_HEAD>(a, ga, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
+          fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
         }
         tc_fence_before();
         __syncwarp();
@@ -994,7 +1037,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           if (row_ok) {
             const int gg = grow - i * a.G;
             __nv_bfloat16* dst = a.attn + ((size_t)(t.bb * a.Q + i) * H + t.kvh * a.G + gg) * d;
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const float inv = l_run > 0.f ? __fdividef(1.f, l_run) : 0.f;
 #pragma unroll
             for (int e = 0; e < d; e += 8) {
               __nv_bfloat162 hb[4];
@@ -1053,7 +1096,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               acc[4 * e + 3] += w * x.w;
             }
           }
-          const float inv = L > 0.f ? 1.f / L : 0.f;
+          const float inv = L > 0.f ? __fdividef(1.f, L) : 0.f;
           __nv_bfloat16* dst = a.attn + ((size_t)(bb * a.Q + i) * a.H + kvh * a.G + gg) * d + sub * per;
 #pragma unroll
           for (int e = 0; e < per; e += 8) {
