@@ -173,7 +173,7 @@ enum { TL_W0 = 0, TL_W1, TL_X0, TL_X1, TL_M0, TL_M1, TL_E0, TL_E1, TL_S_ACC, TL_
 __device__ __forceinline__ void tl_mark(const FwdArgs& a, int n_ph, int p, int ev) {
   if (a.tl) {
     unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)::"memory");  // not moved across memory operations
     a.tl[((size_t)blockIdx.x * n_ph + p) * TL_EVENTS + ev] = t;
   }
 }
@@ -337,117 +337,174 @@ __device__ inline AttUnit att_unit(const FwdArgs& a, const FwdGeom& g, const int
   return t;
 }
 
+// The epilogues below stage the 128 x 32 accumulator group in shared memory
+// (thread = tile row `row`, v[j] = token j), then re-read it with one thread per
+// (token row, quarter of the tile): lane = token row, warp = quarter for the
+// residual and SwiGLU epilogues (conflict-free 16-byte reads: the staging row
+// stride shifts each row by four banks), four adjacent lanes per token row for
+// the q/k/v epilogue (so a head's sum of squares is two shuffles). Every thread
+// then runs the same short code and stores 16-byte vectors.
+
+// 16 floats -> 8 packed bf16 pairs -> two 16-byte stores
+__device__ __forceinline__ void st_bf16x16(__nv_bfloat16* dst, const float* x) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h2);
+  }
+  uint4* p = reinterpret_cast<uint4*>(dst);
+  p[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  p[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 // Residual epilogue of the O and down projections on 32 token rows [m0, m0+32)
-// of one 128-column tile: h += v; xg = bf16(h * gamma_next); partial sum of h^2
-// over the tile's 128 columns per row -> ss[nt][m]. Thread = output column `row`.
-// With h_in_v the old h is already part of v (added by the contributor that holds
-// the tile's last k-chunk, early in its range, so no h load sits on the path).
+// of one 128-column tile: h += v; xg = bf16(h * gamma_next); sum of h^2 over the
+// tile's 128 columns per row -> ss[nt][m]. With h_in_v the old h is already part
+// of v (added by the contributor that holds the tile's last k-chunk, early in its
+// range, so no h load sits on the path). gam_t: the next norm's gains of this
+// tile's 128 columns (shared memory when staged). Uses epi[32 * kEpiStride + 128)
+// for the per-quarter sums.
 __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
-                                                   int m_valid, const float* gam, float* epi, bool h_in_v) {
+                                                   int m_valid, const float* gam_t, float* epi, bool h_in_v) {
   const int D = a.D;
-  const int f = nt * 128 + row;
-  const float gf = gam[f];
-  float hv[32];
+  if (h_in_v) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    hv[j] = (!h_in_v && m0 + j < m_valid) ? __ldcg(a.h + (size_t)(m0 + j) * D + f) : 0.f;
+    for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+  } else {
+    float hv[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (m0 + j < m_valid) {
-      hv[j] += v[j];
-      a.h[(size_t)(m0 + j) * D + f] = hv[j];
-      a.xg[(size_t)(m0 + j) * D + f] = __float2bfloat16(hv[j] * gf);
-    }
-    epi[j * kEpiStride + row] = hv[j] * hv[j];
+    for (int j = 0; j < 32; ++j)
+      hv[j] = m0 + j < m_valid ? __ldcg(a.h + (size_t)(m0 + j) * D + nt * 128 + row) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j] + hv[j];
   }
   named_bar_sync(1, 128);
-  {
-    const int t = threadIdx.x - 64;
-    const int j = t >> 2, q = t & 3;
-    float s = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) s += epi[j * kEpiStride + q * 32 + i];
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    if (q == 0 && m0 + j < m_valid) a.ss[(size_t)nt * a.ss_ld + m0 + j] = s;
+  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
+  const float* src = epi + j * kEpiStride + qq * 32;
+  float y[32];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 f4 = *reinterpret_cast<const float4*>(src + 4 * c);
+    y[4 * c] = f4.x;
+    y[4 * c + 1] = f4.y;
+    y[4 * c + 2] = f4.z;
+    y[4 * c + 3] = f4.w;
+  }
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    s0 += y[i] * y[i];
+    s1 += y[i + 1] * y[i + 1];
+    s2 += y[i + 2] * y[i + 2];
+    s3 += y[i + 3] * y[i + 3];
+  }
+  float* qsum = epi + 32 * kEpiStride;
+  qsum[qq * 32 + j] = (s0 + s1) + (s2 + s3);
+  if (m0 + j < m_valid) {
+    float4* hp = reinterpret_cast<float4*>(a.h + (size_t)(m0 + j) * D + nt * 128 + qq * 32);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) hp[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+    const float* gq = gam_t + qq * 32;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] *= gq[i];
+    __nv_bfloat16* xp = a.xg + (size_t)(m0 + j) * D + nt * 128 + qq * 32;
+    st_bf16x16(xp, y);
+    st_bf16x16(xp + 16, y + 16);
   }
   named_bar_sync(1, 128);
+  if (t < 32 && m0 + t < m_valid)
+    a.ss[(size_t)nt * a.ss_ld + m0 + t] = ((qsum[t] + qsum[32 + t]) + qsum[64 + t]) + qsum[96 + t];
 }
 
 // Per-phase state of the q/k/v projection epilogue: destination of the block's
-// K/V and the q/k RMSNorm gains of this lane (element lane + 32 k of a head).
+// K/V, the q/k RMSNorm gains (gains[0, d) for q, gains[d, 2d) for k) and the RoPE
+// factors of token rows [0, rope_rows) (both in shared memory; rows past
+// rope_rows read the global table).
 struct QkvCtx {
   __nv_bfloat16 *kdst, *vdst;
   int kv_stride;
-  float gq[4], gk[4];
+  const float* gains;
+  const float2* rope;
+  int rope_rows;
 };
 
 // q/k/v epilogue on 32 token rows [m0, m0+32) of one 128-row tile (one head at
 // d = 128, two at d = 64): per-head RMSNorm of q and k, rotate-half RoPE at the
 // row's absolute position, bf16 store of q (qbuf) and of k, v (cache slot len+i
-// in the verify view, block-scratch row i in the draft view). Warp ew handles
-// token rows ew, ew+4, ...; lane holds elements lane + 32 k of the head. The RoPE
-// factors of all its rows are loaded before the staging barrier (one round trip).
+// in the verify view, block-scratch row i in the draft view). Thread = (token row
+// j, quarter qq): d/32 threads per head, each holding elements [16s, 16s+16) and
+// their RoPE partners [d/2 + 16s, d/2 + 16s + 16).
 template <int D_HEAD>
 __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx& q, const float* v, int row, int m0,
                                                  int nt, int m_valid, float* epi, const int* lens_s) {
-  constexpr int d = D_HEAD, nper = d / 32, half = d / 2;
-  const int lane = threadIdx.x & 31, ew = (threadIdx.x >> 5) - 2;
-  float2 cs[8][nper / 2];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int m = m0 + ew + 4 * r;
-#pragma unroll
-    for (int k = 0; k < nper / 2; ++k)
-      cs[r][k] = m < m_valid ? __ldcg(a.rope + (size_t)m * half + lane + 32 * k) : make_float2(1.f, 0.f);
-  }
+  constexpr int d = D_HEAD, half = d / 2, TPH = d / 32;
 #pragma unroll
   for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
   named_bar_sync(1, 128);
-  const int G = a.H / a.Hkv;
+  const int t = threadIdx.x - 64, j = t >> 2, qq = t & 3;
+  const int hl = qq / TPH, e0 = 16 * (qq % TPH);
+  const int m = m0 + j;
+  const int hh = (nt * 128) / d + hl;  // head index in the fused q|k|v rows
+  const int kind = hh < a.H ? 0 : (hh < a.H + a.Hkv ? 1 : 2);
+  const float* src = epi + j * kEpiStride + hl * d;
+  float x1[16], x2[16];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int j = ew + 4 * r, m = m0 + j;
-    if (m >= m_valid) break;
+  for (int c = 0; c < 4; ++c) {
+    const float4 f1 = *reinterpret_cast<const float4*>(src + e0 + 4 * c);
+    const float4 f2 = *reinterpret_cast<const float4*>(src + half + e0 + 4 * c);
+    x1[4 * c] = f1.x, x1[4 * c + 1] = f1.y, x1[4 * c + 2] = f1.z, x1[4 * c + 3] = f1.w;
+    x2[4 * c] = f2.x, x2[4 * c + 1] = f2.y, x2[4 * c + 2] = f2.z, x2[4 * c + 3] = f2.w;
+  }
+  // sum of squares over the head: own 32 elements, then the other TPH-1 threads
+  // (adjacent lanes); every lane shuffles, whatever its head's kind
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    s0 += x1[i] * x1[i];
+    s1 += x1[i + 1] * x1[i + 1];
+    s2 += x2[i] * x2[i];
+    s3 += x2[i + 1] * x2[i + 1];
+  }
+  float ss = (s0 + s1) + (s2 + s3);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  if (TPH == 4) ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  if (kind < 2) {
+    if (a.qk_norm) {
+      const float rr = rsqrtf(ss * (1.0f / d) + a.eps);
+      const float* g = q.gains + (kind == 0 ? 0 : d);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        x1[i] *= rr * g[e0 + i];
+        x2[i] *= rr * g[half + e0 + i];
+      }
+    }
+    const float2* cs = (m < q.rope_rows ? q.rope : a.rope) + (size_t)m * half + e0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {  // element e pairs with e + d/2
+      const float2 f = m < m_valid ? cs[i] : make_float2(1.f, 0.f);
+      const float y1 = x1[i] * f.x - x2[i] * f.y;
+      const float y2 = x2[i] * f.x + x1[i] * f.y;
+      x1[i] = y1;
+      x2[i] = y2;
+    }
+  }
+  if (m < m_valid) {
     const int bb = m / a.Q, i = m - bb * a.Q;
-#pragma unroll
-    for (int hl = 0; hl < 128 / d; ++hl) {
-      const int hh = (nt * 128) / d + hl;  // head index in the fused q|k|v rows
-      const int kind = hh < a.H ? 0 : (hh < a.H + a.Hkv ? 1 : 2);
-      float x[nper];
-#pragma unroll
-      for (int k = 0; k < nper; ++k) x[k] = epi[j * kEpiStride + hl * d + lane + 32 * k];
-      if (kind < 2) {
-        if (a.qk_norm) {
-          float ss = 0.f;
-#pragma unroll
-          for (int k = 0; k < nper; ++k) ss += x[k] * x[k];
-          ss = warp_sum(ss);
-          const float rr = rsqrtf(ss / (float)d + a.eps);
-#pragma unroll
-          for (int k = 0; k < nper; ++k) x[k] = x[k] * rr * (kind == 0 ? q.gq[k] : q.gk[k]);
-        }
-#pragma unroll
-        for (int k = 0; k < nper / 2; ++k) {  // element e pairs with e + d/2
-          const float x1 = x[k], x2 = x[k + nper / 2];
-          x[k] = x1 * cs[r][k].x - x2 * cs[r][k].y;
-          x[k + nper / 2] = x2 * cs[r][k].x + x1 * cs[r][k].y;
-        }
-      }
-      if (kind == 0) {
-        const int kvh = hh / G, g = hh - kvh * G;
-        __nv_bfloat16* dst = a.qbuf + ((size_t)(bb * a.Hkv + kvh) * (a.Q * G) + i * G + g) * d;
-#pragma unroll
-        for (int k = 0; k < nper; ++k) dst[lane + 32 * k] = __float2bfloat16(x[k]);
-      } else {
-        const int kvh = hh - a.H - (kind == 2 ? a.Hkv : 0);
-        const int slot = a.view == VIEW_DRAFT ? i : lens_s[bb] + i;
-        if (slot >= 0 && slot < q.kv_stride) {
-          __nv_bfloat16* dst = (kind == 1 ? q.kdst : q.vdst) + ((size_t)(bb * a.Hkv + kvh) * q.kv_stride + slot) * d;
-#pragma unroll
-          for (int k = 0; k < nper; ++k) dst[lane + 32 * k] = __float2bfloat16(x[k]);
-        }
-      }
+    __nv_bfloat16* dst = nullptr;
+    if (kind == 0) {
+      const int G = a.H / a.Hkv;
+      const int kvh = hh / G, g = hh - kvh * G;
+      dst = a.qbuf + ((size_t)(bb * a.Hkv + kvh) * (a.Q * G) + i * G + g) * d;
+    } else {
+      const int kvh = hh - a.H - (kind == 2 ? a.Hkv : 0);
+      const int slot = a.view == VIEW_DRAFT ? i : lens_s[bb] + i;
+      if (slot >= 0 && slot < q.kv_stride)
+        dst = (kind == 1 ? q.kdst : q.vdst) + ((size_t)(bb * a.Hkv + kvh) * q.kv_stride + slot) * d;
+    }
+    if (dst) {
+      st_bf16x16(dst + e0, x1);
+      st_bf16x16(dst + half + e0, x2);
     }
   }
   named_bar_sync(1, 128);
@@ -455,24 +512,26 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
 
 // SwiGLU epilogue of the gate/up projection on 32 token rows [m0, m0+32) of one
 // tile: rows 0..63 are the gate rows of features nt*64.., rows 64..127 the matching
-// up rows; act = silu(gate) * up in bf16.
+// up rows; act = silu(gate) * up in bf16. Thread = (token row, 16 features).
 __device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
                                                     int m_valid, float* epi) {
-  // stage the whole 128 x 32 group, then every thread takes one feature for 16 tokens
-  // (all four warps run the same code)
 #pragma unroll
   for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
   named_bar_sync(1, 128);
-  const int f = row & 63, j0 = (row >> 6) * 16;
-  __nv_bfloat16* dst = a.act + (size_t)(m0 + j0) * a.F + nt * 64 + f;
+  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
+  if (m0 + j < m_valid) {
+    const float* src = epi + j * kEpiStride + 16 * qq;
+    float y[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    if (m0 + j0 + j < m_valid) {
-      const float g = epi[(j0 + j) * kEpiStride + f];
-      const float u = epi[(j0 + j) * kEpiStride + 64 + f];
-      // fast reciprocal: an IEEE divide has a slow-path branch per element that serialises the loop
-      dst[(size_t)j * a.F] = __float2bfloat16(__fdividef(g, 1.0f + __expf(-g)) * u);
+    for (int c = 0; c < 4; ++c) {
+      const float4 g4 = *reinterpret_cast<const float4*>(src + 4 * c);
+      const float4 u4 = *reinterpret_cast<const float4*>(src + 64 + 4 * c);
+      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)  // fast reciprocal: an IEEE divide branches per element
+        y[4 * c + i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * u[i];
     }
+    st_bf16x16(a.act + (size_t)(m0 + j) * a.F + nt * 64 + 16 * qq, y);
   }
   named_bar_sync(1, 128);
 }
@@ -511,10 +570,10 @@ __device__ __forceinline__ void fwd_argmax_epilogue(const FwdArgs& a, const floa
 template <int D_HEAD>
 __device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const QkvCtx& qc, const int* lens_s,
                                              int epi_kind, float* v, int row, int m0, int nt, int m_valid, float* epi,
-                                             unsigned long long* red, const float* rstd_s, const float* gam,
+                                             unsigned long long* red, const float* rstd_s, const float* gam_t,
                                              bool h_in_v = false) {
   if (epi_kind == EPI_RESID) {
-    fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam, epi, h_in_v);
+    fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam_t, epi, h_in_v);
     return;
   }
 #pragma unroll
@@ -711,20 +770,33 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         named_bar_sync(1, 128);
       }
+      const int first_tile = (int)(u0 / kc), last_tile = (int)((u1 - 1) / kc);
+      // Per-phase epilogue inputs are copied to the attention Q region (unused by
+      // projection phases) at the phase start, off the path of the last tiles:
+      // QKV: q/k norm gains and RoPE rows; O / DOWN: the next norm's gains of the
+      // CTA's tiles.
+      float* stg = reinterpret_cast<float*>(scr - (size_t)128 * d * 2);
+      const int stg_floats = 64 * d;
       const float* gam = nullptr;
+      bool gam_staged = false;
       QkvCtx qc;
       qc.kdst = qc.vdst = nullptr;
       qc.kv_stride = 0;
+      qc.gains = stg;
+      qc.rope = reinterpret_cast<const float2*>(stg + 2 * d);
+      qc.rope_rows = 0;
       if (kind == PH_QKV) {
         const bool dv = a.view == VIEW_DRAFT;
         const float* gq = dv ? a.norms[l].wd_q_norm : a.norms[l].q_norm;
         const float* gk = dv ? a.norms[l].wd_k_norm : a.norms[l].k_norm;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const bool in = a.qk_norm && k < d / 32;
-          qc.gq[k] = in ? gq[lane + 32 * k] : 1.f;
-          qc.gk[k] = in ? gk[lane + 32 * k] : 1.f;
+        for (int i = et; i < d; i += 128) {
+          stg[i] = a.qk_norm ? gq[i] : 1.f;
+          stg[d + i] = a.qk_norm ? gk[i] : 1.f;
         }
+        qc.rope_rows = min(a.M, (stg_floats - 2 * d) / d);  // a row is d/2 float2
+        const float4* rs = reinterpret_cast<const float4*>(a.rope);
+        float4* rd = reinterpret_cast<float4*>(stg + 2 * d);
+        for (int i = et; i < qc.rope_rows * (d / 4); i += 128) rd[i] = __ldcg(rs + i);
         if (dv) {
           const size_t lo = (size_t)l * a.batch * a.Hkv * a.max_block * d;
           qc.kdst = a.blk_k + lo;
@@ -736,12 +808,19 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           qc.vdst = a.vc + lo;
           qc.kv_stride = a.cap;
         }
-      } else if (kind == PH_O) {
-        gam = a.norms[l].mlp_norm;
-      } else if (kind == PH_DOWN) {
-        gam = l + 1 < a.L ? a.norms[l + 1].attn_norm : a.final_norm;
+      } else if (kind == PH_O || kind == PH_DOWN) {
+        gam = kind == PH_O ? a.norms[l].mlp_norm : (l + 1 < a.L ? a.norms[l + 1].attn_norm : a.final_norm);
+        const int n = (last_tile - first_tile + 1) * 128;
+        if (n <= stg_floats) {
+          for (int i = et; i < n; i += 128) stg[i] = gam[(size_t)first_tile * 128 + i];
+          gam_staged = true;
+        }
       }
-      const int first_tile = (int)(u0 / kc);
+      named_bar_sync(1, 128);
+      auto gam_tile = [&](int t) -> const float* {
+        if (!gam) return nullptr;
+        return gam_staged ? stg + (t - first_tile) * 128 : gam + (size_t)t * 128;
+      };
       const int m_valid = min(a.Mt, a.M);
       // owner of unit uu = the CTA whose non-empty range holds it (largest c with start <= uu)
       auto owner = [&](int uu) {
@@ -812,7 +891,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_after();
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
-            fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam);
+            fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam_tile(nt));
           }
           tc_fence_before();
           __syncwarp();
@@ -907,7 +986,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             add4(v, x);
           }
           if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
-          fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam, true);
+          fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam_tile(nt), true);
         }
         tc_fence_before();
         __syncwarp();
