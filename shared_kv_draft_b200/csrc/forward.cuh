@@ -678,7 +678,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
     if (et == 0) {
       const int tgt = phase_target(a, g, dep);
       const int code = wait_count_code(a.phase_cnt + dep, tgt, a.status, a.poll_ns);
-      fwd_diag(a, code, 12, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
+      if (code == -1) fwd_diag(a, code, 12, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
       r = code == 1;
     }
     r = bcast(r);
@@ -954,7 +954,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         bool ready = false;
         if (et == 0) {
           const int code = wait_count_code(a.tile_cnt + t, n_contrib - 1, a.status);
-          fwd_diag(a, code, 17, p, it, t, n_contrib, *(volatile int*)(a.tile_cnt + t));
+          if (code == -1) fwd_diag(a, code, 17, p, it, t, n_contrib, *(volatile int*)(a.tile_cnt + t));
           ready = code == 1;
           if (ready) a.tile_cnt[t] = 0;
         }
