@@ -170,7 +170,11 @@ __device__ inline void fwd_diag(const FwdArgs& a, int code, int site, int p, int
 //   stored, arrival counted, partials loaded, epilogue done, completion signalled.
 enum { TL_W0 = 0, TL_W1, TL_X0, TL_X1, TL_M0, TL_M1, TL_E0, TL_E1, TL_S_ACC, TL_S_PART, TL_S_CNT, TL_S_LOAD,
        TL_S_EPI, TL_S_SIG, TL_R0, TL_R1, TL_EVENTS };
+// The marks exist only in the profiling instantiation of the kernel (TL = true):
+// their address arithmetic and stores change register allocation around them.
+template <bool TL>
 __device__ __forceinline__ void tl_mark(const FwdArgs& a, int n_ph, int p, int ev) {
+  if constexpr (!TL) return;
   if (a.tl) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)::"memory");  // not moved across memory operations
@@ -638,7 +642,7 @@ __device__ inline void fwd_finalize(const FwdArgs& a, int n_ph) {
 }
 
 // Epilogue warps (2-5) of the persistent forward kernel.
-template <int D_HEAD>
+template <int D_HEAD, bool TL>
 __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeom& g, uint8_t* smem,
                                                   uint32_t stage_bytes, int S, uint8_t* scr,
                                                   unsigned long long* red, float* rstd_s, const int* lens_s,
@@ -716,7 +720,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       // ---------------- embedding rows ----------------
       const float* g0 = a.norms[0].attn_norm;
       const int parts = D / 128;
-      if (et == 0 && c < a.M) tl_mark(a, n_ph, p, TL_E0);
+      if (et == 0 && c < a.M) tl_mark<TL>(a, n_ph, p, TL_E0);
       for (int m = c; m < a.M; m += Gd) {
         const int bb = m / a.Q, i = m - bb * a.Q;
         int id;
@@ -760,7 +764,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         ok = false;
         break;
       }
-      if (et == 0) tl_mark(a, n_ph, p, TL_E0);
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E0);
       if (kind == PH_QKV || kind == PH_GU || kind == PH_LM) {
         if (et < a.Mt) {
           float s = 0.f;
@@ -887,7 +891,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             ok = false;
             break;
           }
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
+          if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_ACC);
           tc_fence_after();
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             tmem_ld32(taddr + m0, v);
@@ -896,9 +900,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acce[buf]);
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
+          if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_EPI);
           signal(p);
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
+          if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_SIG);
           continue;
         }
         const int c_lo = owner(t * kc), c_hi = owner((t + 1) * kc - 1);
@@ -913,7 +917,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             ok = false;
             break;
           }
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
+          if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_ACC);
           tc_fence_after();
           const bool add_h = gp.epi == EPI_RESID && c == c_hi;
           // partial slot layout [token m / 4][weight row][m % 4]: a thread moves float4s and a
@@ -941,7 +945,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           __syncwarp();
           if (lane == 0) mbar_arrive(&acce[buf]);
           named_bar_sync(1, 128);
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_PART);
+          if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_PART);
           if (et == 0) red_release_gpu_add(a.tile_cnt + t, 1);
           continue;
         }
@@ -958,7 +962,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           ready = code == 1;
           if (ready) a.tile_cnt[t] = 0;
         }
-        if (et == 0) tl_mark(a, n_ph, p, TL_S_CNT);
+        if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_CNT);
         if (!bcast(ready)) {
           ok = false;
           break;
@@ -971,7 +975,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           ok = false;
           break;
         }
-        if (et == 0) tl_mark(a, n_ph, p, TL_S_ACC);
+        if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_ACC);
         tc_fence_after();
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
           tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
@@ -985,18 +989,18 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             load4(x, s0, s1, s2, s3, m0);
             add4(v, x);
           }
-          if (et == 0) tl_mark(a, n_ph, p, TL_S_LOAD);
+          if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_LOAD);
           fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam_tile(nt), true);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[buf]);
-        if (et == 0) tl_mark(a, n_ph, p, TL_S_EPI);
+        if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_EPI);
         signal(p);
-        if (et == 0) tl_mark(a, n_ph, p, TL_S_SIG);
+        if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_SIG);
       }
       it += (int)(u1 - u0);
-      if (et == 0) tl_mark(a, n_ph, p, TL_E1);
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E1);
     } else if (kind == PH_ATTN) {
       // ---------------- block attention (thread = query row of the tile) ----------------
       if (c >= g.att_units) continue;
@@ -1004,7 +1008,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         ok = false;
         break;
       }
-      if (et == 0) tl_mark(a, n_ph, p, TL_E0);
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E0);
       for (int u = c; ok && u < g.att_units; u += Gd) {
         const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
         const int grow = t.r * 128 + row;
@@ -1027,7 +1031,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             ok = false;
             break;
           }
-          if (et == 0) tl_mark(a, n_ph, p, j == 0 ? TL_R0 : TL_S_ACC);  // score tile ready
+          if (et == 0) tl_mark<TL>(a, n_ph, p, j == 0 ? TL_R0 : TL_S_ACC);  // score tile ready
           tc_fence_after();
           const int key0 = t.key_lo + j * 64;
           float sv[64];
@@ -1039,7 +1043,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             if (key0 + tt < lim) mx = fmaxf(mx, sv[tt] * a.scale_log2);
           const float m_new = fmaxf(m_run, mx);
           const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
-          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_PART);  // row maxima done
+          if (j == 0 && et == 0) tl_mark<TL>(a, n_ph, p, TL_S_PART);  // row maxima done
           if (j > 0) {
             // the previous tile's P V must be complete before O is rescaled
             if (!bar_wait_all(o_full, (uint32_t)(ta - 1) & 1u, 15)) {
@@ -1097,7 +1101,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(p_full);
-          if (j == 0 && et == 0) tl_mark(a, n_ph, p, TL_S_CNT);  // P written
+          if (j == 0 && et == 0) tl_mark<TL>(a, n_ph, p, TL_S_CNT);  // P written
         }
         if (!ok) break;
         // the unit's last P V, then O into registers
@@ -1110,7 +1114,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
 #pragma unroll
         for (int c0 = 0; c0 < d; c0 += 32) tmem_ld32(tO + lane_base + c0, o + c0);
         tc_fence_before();
-        if (et == 0) tl_mark(a, n_ph, p, TL_R1);
+        if (et == 0) tl_mark<TL>(a, n_ph, p, TL_R1);
         const int H = a.H;
         if (t.n_chunks == 1) {
           if (row_ok) {
@@ -1135,7 +1139,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         signal(p);
       }
-      if (et == 0) tl_mark(a, n_ph, p, TL_E1);
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E1);
     } else if (kind == PH_COMBINE) {
       // ---------------- merge of key-chunk partials ----------------
       if (c >= g.comb_units) continue;
@@ -1143,7 +1147,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         ok = false;
         break;
       }
-      if (et == 0) tl_mark(a, n_ph, p, TL_E0);
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E0);
       constexpr int per = d / 8;  // columns per thread: thread et takes row et % 16 and column block et / 16
       for (int u = c; u < g.comb_units; u += Gd) {
         const int slot = u / (128 / kCombineRows), grp = u % (128 / kCombineRows);
@@ -1187,7 +1191,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         signal(p);
       }
-      if (et == 0) tl_mark(a, n_ph, p, TL_E1);
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E1);
     }
   }
 }
@@ -1196,7 +1200,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
 
 namespace orthrus {
 
-template <int D_HEAD>
+template <int D_HEAD, bool TL>
 __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_constant__ FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1319,7 +1323,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
           const long long W = gp.units;
           const long long u0 = unit_start(W, Gd, c), u1 = unit_start(W, Gd, c + 1);
           const int kc = gp.k_chunks;
-          if (u0 < u1 && wprod) tl_mark(a, n_ph, p, TL_W0);
+          if (u0 < u1 && wprod) tl_mark<TL>(a, n_ph, p, TL_W0);
           for (long long u = u0; u < u1; ++u, ++it) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -1345,13 +1349,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 ok = false;
                 break;
               }
-              if (u == u0) tl_mark(a, n_ph, p, TL_X0);
+              if (u == u0) tl_mark<TL>(a, n_ph, p, TL_X0);
               mbar_arrive_expect_tx(&full[s], x_bytes);
               tma_load_3d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k);
             }
             last_ph[s] = (int)ph;
           }
-          if (u0 < u1) tl_mark(a, n_ph, p, wprod ? TL_W1 : TL_X1);
+          if (u0 < u1) tl_mark<TL>(a, n_ph, p, wprod ? TL_W1 : TL_X1);
         } else if (kind == PH_ATTN) {
           for (int u = c; ok && u < g.att_units; u += Gd, ++qu) {
             const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
@@ -1466,7 +1470,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 ok = false;
                 break;
               }
-              if (u == u0) tl_mark(a, n_ph, p, TL_M0);
+              if (u == u0) tl_mark<TL>(a, n_ph, p, TL_M0);
               tc_fence_after();
               const uint32_t wa = smem_u32(stage_ptr(s));
               const uint32_t xa = wa + 32768;
@@ -1484,7 +1488,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
             mma_commit(&accf[buf]);
             ++seg;
           }
-          if (u0 < u1) tl_mark(a, n_ph, p, TL_M1);
+          if (u0 < u1) tl_mark<TL>(a, n_ph, p, TL_M1);
         } else if (kind == PH_ATTN) {
           const uint32_t qa = smem_u32(sQ);
           for (int u = c; ok && u < g.att_units; u += Gd, ++qu) {
@@ -1542,7 +1546,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
     }
   } else {
     // ======================= epilogue warps =======================
-    fwd_epilogue_role<D_HEAD>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, ust_s, accf, acce, full,
+    fwd_epilogue_role<D_HEAD, TL>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, ust_s, accf, acce, full,
                               s_full, p_full, o_full, flag, tmem_base, tS, tO);
   }
 

@@ -504,14 +504,27 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
+  // the timeline instantiation only while a timeline buffer is set (profiling)
   if (c.head_dim == 128) {
-    static bool set = false;
-    if (!set) set = set_smem_attr(forward_kernel<128>, kSmemLimit);
-    e = cudaLaunchKernelEx(&cfg, forward_kernel<128>, a);
+    if (a.tl) {
+      static bool set = false;
+      if (!set) set = set_smem_attr(forward_kernel<128, true>, kSmemLimit);
+      e = cudaLaunchKernelEx(&cfg, forward_kernel<128, true>, a);
+    } else {
+      static bool set = false;
+      if (!set) set = set_smem_attr(forward_kernel<128, false>, kSmemLimit);
+      e = cudaLaunchKernelEx(&cfg, forward_kernel<128, false>, a);
+    }
   } else {
-    static bool set = false;
-    if (!set) set = set_smem_attr(forward_kernel<64>, kSmemLimit);
-    e = cudaLaunchKernelEx(&cfg, forward_kernel<64>, a);
+    if (a.tl) {
+      static bool set = false;
+      if (!set) set = set_smem_attr(forward_kernel<64, true>, kSmemLimit);
+      e = cudaLaunchKernelEx(&cfg, forward_kernel<64, true>, a);
+    } else {
+      static bool set = false;
+      if (!set) set = set_smem_attr(forward_kernel<64, false>, kSmemLimit);
+      e = cudaLaunchKernelEx(&cfg, forward_kernel<64, false>, a);
+    }
   }
   return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }

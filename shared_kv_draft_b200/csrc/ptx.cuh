@@ -101,7 +101,7 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t pari
 #pragma unroll 1
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 1023u) == 0u) {
+    if ((it & 1023u) == 1023u) {  // status / clock checks off the first polls
       if (*(volatile int*)status != 0) return false;
       if (clock64() - t0 > kWaitLimitCycles) {
         set_status(status, ORTHRUS_ERR_TIMEOUT);
@@ -135,7 +135,7 @@ __device__ __forceinline__ int mbar_wait_code(uint64_t* bar, uint32_t parity, in
 #pragma unroll 1
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return 1;
-    if ((it & 15u) == 0u) {
+    if ((it & 15u) == 15u) {
       if (*(volatile int*)status != 0) return 0;
       if (clock64() - t0 > kWaitLimitCycles) {
         set_status(status, ORTHRUS_ERR_TIMEOUT);
@@ -207,7 +207,7 @@ __device__ __forceinline__ int wait_count_code(const int* cnt, int target, int* 
   for (uint32_t it = 0;; ++it) {
     sleep_ns(poll_ns);
     if (ld_acquire_gpu(cnt) >= target) return 1;
-    if ((it & 255u) == 0u) {
+    if ((it & 255u) == 255u) {
       if (*(volatile int*)status != 0) return 0;
       if (clock64() - t0 > kWaitLimitCycles) {
         set_status(status, ORTHRUS_ERR_TIMEOUT);
