@@ -409,9 +409,12 @@ __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float
     float4* hp = reinterpret_cast<float4*>(a.h + (size_t)(m0 + j) * D + nt * 128 + qq * 32);
 #pragma unroll
     for (int c = 0; c < 8; ++c) hp[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
-    const float* gq = gam_t + qq * 32;
+    const float4* gq = reinterpret_cast<const float4*>(gam_t + qq * 32);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] *= gq[i];
+    for (int c = 0; c < 8; ++c) {
+      const float4 g4 = gq[c];
+      y[4 * c] *= g4.x, y[4 * c + 1] *= g4.y, y[4 * c + 2] *= g4.z, y[4 * c + 3] *= g4.w;
+    }
     __nv_bfloat16* xp = a.xg + (size_t)(m0 + j) * D + nt * 128 + qq * 32;
     st_bf16x16(xp, y);
     st_bf16x16(xp + 16, y + 16);
@@ -476,21 +479,39 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
   if (kind < 2) {
     if (a.qk_norm) {
       const float rr = rsqrtf(ss * (1.0f / d) + a.eps);
-      const float* g = q.gains + (kind == 0 ? 0 : d);
+      const float4* g1 = reinterpret_cast<const float4*>(q.gains + (kind == 0 ? 0 : d) + e0);
+      const float4* g2 = g1 + half / 4;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        x1[i] *= rr * g[e0 + i];
-        x2[i] *= rr * g[half + e0 + i];
+      for (int c = 0; c < 4; ++c) {
+        const float4 a1 = g1[c], a2 = g2[c];
+        x1[4 * c] *= rr * a1.x, x1[4 * c + 1] *= rr * a1.y, x1[4 * c + 2] *= rr * a1.z, x1[4 * c + 3] *= rr * a1.w;
+        x2[4 * c] *= rr * a2.x, x2[4 * c + 1] *= rr * a2.y, x2[4 * c + 2] *= rr * a2.z, x2[4 * c + 3] *= rr * a2.w;
       }
     }
-    const float2* cs = (m < q.rope_rows ? q.rope : a.rope) + (size_t)m * half + e0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {  // element e pairs with e + d/2
-      const float2 f = m < m_valid ? cs[i] : make_float2(1.f, 0.f);
-      const float y1 = x1[i] * f.x - x2[i] * f.y;
-      const float y2 = x2[i] * f.x + x1[i] * f.y;
+    // element e pairs with e + d/2
+    auto rot = [&](int i, float c, float sn) {
+      const float y1 = x1[i] * c - x2[i] * sn;
+      const float y2 = x2[i] * c + x1[i] * sn;
       x1[i] = y1;
       x2[i] = y2;
+    };
+    if (m < q.rope_rows) {
+      // staged rows: 16-byte chunk c of segment s sits at chunk s*8 + ((c + 2s + (m & 1)) & 7) of the row
+      // (the eight lanes of one shared-memory wavefront then hit eight different bank groups)
+      const int sg = e0 / 16;
+      const float4* rp = reinterpret_cast<const float4*>(q.rope + (size_t)m * half) + sg * 8;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 f = rp[(c + 2 * sg + (m & 1)) & 7];
+        rot(2 * c, f.x, f.y);
+        rot(2 * c + 1, f.z, f.w);
+      }
+    } else if (m < m_valid) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 f = a.rope[(size_t)m * half + e0 + i];
+        rot(i, f.x, f.y);
+      }
     }
   }
   if (m < m_valid) {
@@ -797,10 +818,13 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           stg[i] = a.qk_norm ? gq[i] : 1.f;
           stg[d + i] = a.qk_norm ? gk[i] : 1.f;
         }
-        qc.rope_rows = min(a.M, (stg_floats - 2 * d) / d);  // a row is d/2 float2
+        qc.rope_rows = min(a.M, (stg_floats - 2 * d) / d);  // a row is d/2 float2 = d/4 16-byte chunks
         const float4* rs = reinterpret_cast<const float4*>(a.rope);
         float4* rd = reinterpret_cast<float4*>(stg + 2 * d);
-        for (int i = et; i < qc.rope_rows * (d / 4); i += 128) rd[i] = __ldcg(rs + i);
+        for (int i = et; i < qc.rope_rows * (d / 4); i += 128) {
+          const int m = i / (d / 4), k = i - m * (d / 4), sg = k >> 3, cc = k & 7;
+          rd[m * (d / 4) + sg * 8 + ((cc + 2 * sg + (m & 1)) & 7)] = __ldcg(rs + i);
+        }
         if (dv) {
           const size_t lo = (size_t)l * a.batch * a.Hkv * a.max_block * d;
           qc.kdst = a.blk_k + lo;
