@@ -90,7 +90,7 @@ constexpr int kPhasesPerLayer = 6;  // QKV, ATTN, COMBINE, O, GU, DOWN
 constexpr int kFwdThreads = 224;
 constexpr int kMaxStages = 16;
 constexpr int kMaxSlots = 256;        // attention (sequence, kv head, row tile) slots per launch
-constexpr int kMaxChunks = 18;        // key chunks per slot (16 cache chunks + draft block + slack)
+constexpr int kMaxChunks = 34;        // key chunks per slot (32 cache chunks + draft block + slack)
 constexpr int kCombineRows = 16;      // rows per merge unit
 constexpr int kScratchBytes = 17408;  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
 constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers
@@ -109,7 +109,7 @@ struct FwdArgs {
   int nb, Q, M, Mt, mt_idx, stages, cap, max_block, batch;
   int lookahead;             // weight tiles the weight producer loads ahead of a phase's input dependency
   int poll_ns;               // sleep between polls of a phase counter
-  int ck;                    // keys per attention chunk: fixed per plan (multiple of 64, >= capacity / 16),
+  int ck;                    // keys per attention chunk: fixed per plan (multiple of 64, >= capacity / 32),
                              // so a row's softmax runs over the same absolute key chunks whatever
                              // the block size: verify rows equal the plain AR rows bit for bit
   const int* pending;        // [nb]

@@ -778,8 +778,8 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->ss = (float*)(base + wl.ss);
   P->ss_ld = wl.ss_ld;
   P->mega_slots = wl.mega_slots;
-  // attention chunk of the persistent kernel: at most 16 chunks over the whole capacity
-  P->fwd_ck = std::max(64, round_up((P->cap + 15) / 16, 64));
+  // attention chunk of the persistent kernel: at most kMaxChunks - 2 chunks over the whole capacity
+  P->fwd_ck = std::max(64, round_up((P->cap + kMaxChunks - 3) / (kMaxChunks - 2), 64));
   P->fwd_ck = std::max(P->fwd_ck, round_up(env_int("ORTHRUS_ATT_CK", 0), 64));
   P->fwd_att_o = (float*)(base + wl.fwd_att_o);
   P->fwd_att_ml = (float2*)(base + wl.fwd_att_ml);
