@@ -706,11 +706,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       if (code == -1) fwd_diag(a, code, 12, cur_p, it, dep, tgt, *(volatile int*)(a.phase_cnt + dep));
       r = code == 1;
     }
+    // thread 0's acquire, then the barrier in bcast: the other threads' later
+    // reads are ordered after the released writes (happens-before is transitive)
     r = bcast(r);
-    if (r) {
-      (void)ld_acquire_gpu(a.phase_cnt + dep);
-      acq = dep;
-    }
+    if (r) acq = dep;
     return r;
   };
   // outputs of a completion unit written -> count it (the barrier orders the other

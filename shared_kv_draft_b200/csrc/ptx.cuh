@@ -197,9 +197,19 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 __device__ __forceinline__ void sleep_ns(uint32_t ns) { asm volatile("nanosleep.u32 %0;" ::"r"(ns)); }
 
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // Wait until *cnt >= target (acquire). False once the status word holds an
 // error or after about 2 s (then ORTHRUS_ERR_TIMEOUT is recorded).
 // 1 = reached, 0 = gave up because the status word holds an error, -1 = timed out here.
+// One load in flight at a time: every CTA polls the same few counters, and more
+// polls in flight slow the L2 slice that holds them, weight stream included.
 __device__ __forceinline__ int wait_count_code(const int* cnt, int target, int* status, uint32_t poll_ns = 64) {
   if (ld_acquire_gpu(cnt) >= target) return 1;
   const long long t0 = clock64();
