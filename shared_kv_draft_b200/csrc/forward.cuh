@@ -563,31 +563,51 @@ __device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const floa
 
 // Greedy head of the LM projection on 32 token rows [m0, m0+32) of one 128-row
 // vocabulary tile: optional fp32 logits, NaN check, and the running argmax key of
-// each token row (max over the tile's rows, then one atomic per row).
+// each token row. Thread = (token row, 32 vocabulary rows): the max over its 32
+// keys, then over the four quarters, then one atomic per token row.
 __device__ __forceinline__ void fwd_argmax_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
-                                                    int m_valid, unsigned long long* red) {
-  const int ew = (threadIdx.x >> 5) - 2, lane = threadIdx.x & 31;
-  const uint32_t col = nt * 128 + row;  // vocabulary index
+                                                    int m_valid, float* epi, unsigned long long* red) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int m = m0 + j;
-    unsigned long long key = 0ull;
-    if (m < m_valid) {
-      if (a.logits) a.logits[(size_t)m * a.V + col] = v[j];
-      if (isnan(v[j])) set_status(a.status, ORTHRUS_ERR_NAN);
-      else key = argmax_key(v[j], col);
+  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+  named_bar_sync(1, 128);
+  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
+  const int m = m0 + j;
+  unsigned long long best = 0ull;
+  if (m < m_valid) {
+    const float* src = epi + j * kEpiStride + qq * 32;
+    float y[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 f4 = *reinterpret_cast<const float4*>(src + 4 * c);
+      y[4 * c] = f4.x, y[4 * c + 1] = f4.y, y[4 * c + 2] = f4.z, y[4 * c + 3] = f4.w;
     }
+    const uint32_t col0 = nt * 128 + qq * 32;  // vocabulary index of y[0]
+    bool bad = false;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) key = ull_max(key, __shfl_xor_sync(0xffffffffu, key, o));
-    if (lane == 0) red[ew * 32 + j] = key;
+    for (int i = 0; i < 32; ++i) {
+      const bool nan = isnan(y[i]);
+      bad |= nan;
+      best = ull_max(best, nan ? 0ull : argmax_key(y[i], col0 + i));
+    }
+    if (bad) set_status(a.status, ORTHRUS_ERR_NAN);
+    if (a.logits) {
+      float* lp = a.logits + (size_t)m * a.V + col0;
+      if ((a.V & 3) == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          reinterpret_cast<float4*>(lp)[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) lp[i] = y[i];
+      }
+    }
   }
+  red[qq * 32 + j] = best;
   named_bar_sync(1, 128);
-  if (ew == 0) {
-    const int m = m0 + lane;
-    const unsigned long long k = ull_max(ull_max(red[lane], red[32 + lane]), ull_max(red[64 + lane], red[96 + lane]));
-    if (m < m_valid && k != 0ull) atomicMax(a.amax + m, k);
+  if (t < 32 && m0 + t < m_valid) {
+    const unsigned long long k = ull_max(ull_max(red[t], red[32 + t]), ull_max(red[64 + t], red[96 + t]));
+    if (k != 0ull) atomicMax(a.amax + m0 + t, k);
   }
-  named_bar_sync(1, 128);
 }
 
 // Epilogue of one 32-row group for the GEMM phase kinds. Consumers of a
@@ -605,7 +625,7 @@ __device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const QkvCtx& qc,
   for (int j = 0; j < 32; ++j) v[j] *= rstd_s[m0 + j];
   if (epi_kind == EPI_QKV) fwd_qkv_epilogue<D_HEAD>(a, qc, v, row, m0, nt, m_valid, epi, lens_s);
   else if (epi_kind == EPI_SWIGLU) fwd_swiglu_epilogue(a, v, row, m0, nt, m_valid, epi);
-  else fwd_argmax_epilogue(a, v, row, m0, nt, m_valid, red);
+  else fwd_argmax_epilogue(a, v, row, m0, nt, m_valid, epi, red);
 }
 
 }  // namespace orthrus
