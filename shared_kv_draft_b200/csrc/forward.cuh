@@ -1077,13 +1077,25 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           if (et == 0) tl_mark<TL>(a, n_ph, p, j == 0 ? TL_R0 : TL_S_ACC);  // score tile ready
           tc_fence_after();
           const int key0 = t.key_lo + j * 64;
-          float sv[64];
-          tmem_ld32(tS + lane_base, sv);
-          tmem_ld32(tS + lane_base + 32, sv + 32);
-          float mx = -INFINITY;
+          const int nv = min(max(lim - key0, 0), 64);  // keys of this tile the row sees
+          // Row maximum over the visible scores: two 32-column loads, four independent
+          // chains (the scale is positive, so max(s) * scale = max(s * scale) exactly).
+          // The scores are loaded again for the exponentials below rather than held:
+          // fewer live registers leave room for independent work in both passes.
+          float sv[32];
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-          for (int tt = 0; tt < 64; ++tt)
-            if (key0 + tt < lim) mx = fmaxf(mx, sv[tt] * a.scale_log2);
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            tmem_ld32(tS + lane_base + c0, sv);
+#pragma unroll
+            for (int tt = 0; tt < 32; tt += 4) {
+              mx0 = fmaxf(mx0, c0 + tt < nv ? sv[tt] : -INFINITY);
+              mx1 = fmaxf(mx1, c0 + tt + 1 < nv ? sv[tt + 1] : -INFINITY);
+              mx2 = fmaxf(mx2, c0 + tt + 2 < nv ? sv[tt + 2] : -INFINITY);
+              mx3 = fmaxf(mx3, c0 + tt + 3 < nv ? sv[tt + 3] : -INFINITY);
+            }
+          }
+          const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * a.scale_log2;
           const float m_new = fmaxf(m_run, mx);
           const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
           if (j == 0 && et == 0) tl_mark<TL>(a, n_ph, p, TL_S_PART);  // row maxima done
@@ -1105,15 +1117,17 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               }
             }
           }
-          float sum = 0.f;
+          float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 32) {
+            tmem_ld32(tS + lane_base + c0, sv);
             uint32_t pk[16];
 #pragma unroll
             for (int tt = 0; tt < 32; tt += 2) {
-              const float p0 = (key0 + c0 + tt < lim) ? fast_exp2(sv[c0 + tt] * a.scale_log2 - m_new) : 0.f;
-              const float p1 = (key0 + c0 + tt + 1 < lim) ? fast_exp2(sv[c0 + tt + 1] * a.scale_log2 - m_new) : 0.f;
-              sum += p0 + p1;
+              const float p0 = (c0 + tt < nv) ? fast_exp2(sv[tt] * a.scale_log2 - m_new) : 0.f;
+              const float p1 = (c0 + tt + 1 < nv) ? fast_exp2(sv[tt + 1] * a.scale_log2 - m_new) : 0.f;
+              sum0 += p0;
+              sum1 += p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
               pk[tt / 2] = *reinterpret_cast<uint32_t*>(&h2);
             }
@@ -1125,7 +1139,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                   make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
             }
           }
-          l_run = l_run * alpha + sum;
+          l_run = l_run * alpha + (sum0 + sum1);
           m_run = m_new;
           // V rows of keys no row may see are zeroed (stale or poisoned cache rows)
           if (key0 + 64 > kv_end && row < 64 && key0 + row >= kv_end) {
