@@ -74,7 +74,9 @@ typedef struct {
 } orthrus_config;
 
 /* Device pointers to the weights. Per-layer members are HOST arrays of
- * n_layers DEVICE pointers. Norm gains are fp32; matrices are bf16.
+ * n_layers DEVICE pointers. Norm gains are fp32; matrices are bf16. Every
+ * pointer is 16-byte aligned (tensor-map bases; norm gains are read as
+ * 16-byte vectors); orthrus_plan_init returns ORTHRUS_ERR_ARG otherwise.
  * wd_* are the draft attention module's own projections and q/k norm gains;
  * the draft view reuses attn_norm, mlp_norm, the MLP, final_norm and lm_head. */
 typedef struct {

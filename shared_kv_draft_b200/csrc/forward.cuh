@@ -147,7 +147,7 @@ struct FwdArgs {
 
 // Records the first wait that ran out of time: site, phase, ring position and
 // two site-specific values (diag[0] = 1 once written).
-__device__ inline void fwd_diag(const FwdArgs& a, int code, int site, int p, int it, int x0 = 0, int x1 = 0,
+__device__ __noinline__ void fwd_diag(const FwdArgs& a, int code, int site, int p, int it, int x0 = 0, int x1 = 0,
                                 int x2 = 0) {
   if (code != -1 || !a.diag) return;
   if (atomicCAS(a.diag, 0, 1) != 0) return;
@@ -800,25 +800,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       if (u0 == u1) continue;
       // unit-range start of every CTA (W * Gd < 2^31 for every phase shape accepted)
       for (int i = et; i <= Gd; i += 128) ust_s[i] = (int)(((long long)W * i) / Gd);
-      if (!acquire_phase(dep)) {
-        ok = false;
-        break;
-      }
-      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E0);
-      if (kind == PH_QKV || kind == PH_GU || kind == PH_LM) {
-        if (et < a.Mt) {
-          float s = 0.f;
-          if (et < a.M)
-            for (int pp = 0; pp < D / 128; ++pp) s += __ldcg(a.ss + (size_t)pp * a.ss_ld + et);
-          rstd_s[et] = et < a.M ? rsqrtf(s / (float)D + a.eps) : 0.f;
-        }
-        named_bar_sync(1, 128);
-      }
       const int first_tile = (int)(u0 / kc), last_tile = (int)((u1 - 1) / kc);
       // Per-phase epilogue inputs are copied to the attention Q region (unused by
-      // projection phases) at the phase start, off the path of the last tiles:
-      // QKV: q/k norm gains and RoPE rows; O / DOWN: the next norm's gains of the
-      // CTA's tiles.
+      // projection phases): QKV: q/k norm gains and RoPE rows; O / DOWN: the next norm's
+      // gains of the CTA's tiles. Weights are copied before the previous phase is
+      // awaited (RoPE rows too, once EMBED is long done), each thread's loads all in
+      // flight before its shared-memory stores.
       float* stg = reinterpret_cast<float*>(scr - (size_t)128 * d * 2);
       const int stg_floats = 64 * d;
       const float* gam = nullptr;
@@ -829,21 +816,40 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       qc.gains = stg;
       qc.rope = reinterpret_cast<const float2*>(stg + 2 * d);
       qc.rope_rows = 0;
-      if (kind == PH_QKV) {
-        const bool dv = a.view == VIEW_DRAFT;
-        const float* gq = dv ? a.norms[l].wd_q_norm : a.norms[l].q_norm;
-        const float* gk = dv ? a.norms[l].wd_k_norm : a.norms[l].k_norm;
-        for (int i = et; i < d; i += 128) {
-          stg[i] = a.qk_norm ? gq[i] : 1.f;
-          stg[d + i] = a.qk_norm ? gk[i] : 1.f;
-        }
-        qc.rope_rows = min(a.M, (stg_floats - 2 * d) / d);  // a row is d/2 float2 = d/4 16-byte chunks
+      // RoPE rows [0, rope_rows) -> shared memory, 16-byte chunk c of segment s at chunk
+      // s*8 + ((c + 2s + (m & 1)) & 7) of the row (conflict-free reads in the epilogue)
+      auto stage_rope = [&]() {
         const float4* rs = reinterpret_cast<const float4*>(a.rope);
         float4* rd = reinterpret_cast<float4*>(stg + 2 * d);
-        for (int i = et; i < qc.rope_rows * (d / 4); i += 128) {
-          const int m = i / (d / 4), k = i - m * (d / 4), sg = k >> 3, cc = k & 7;
-          rd[m * (d / 4) + sg * 8 + ((cc + 2 * sg + (m & 1)) & 7)] = __ldcg(rs + i);
+        const int n = qc.rope_rows * (d / 4);  // a row is d/2 float2 = d/4 16-byte chunks
+        for (int b0 = 0; b0 < n; b0 += 128 * 8) {
+          float4 buf[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = b0 + et + 128 * k;
+            buf[k] = i < n ? __ldcg(rs + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = b0 + et + 128 * k;
+            if (i < n) {
+              const int m = i / (d / 4), kk = i - m * (d / 4), sg = kk >> 3, cc = kk & 7;
+              rd[m * (d / 4) + sg * 8 + ((cc + 2 * sg + (m & 1)) & 7)] = buf[k];
+            }
+          }
         }
+      };
+      if (kind == PH_QKV) {
+        const bool dv = a.view == VIEW_DRAFT;
+        const float4* gq = reinterpret_cast<const float4*>(dv ? a.norms[l].wd_q_norm : a.norms[l].q_norm);
+        const float4* gk = reinterpret_cast<const float4*>(dv ? a.norms[l].wd_k_norm : a.norms[l].k_norm);
+        if (et < d / 2) {  // d/4 float4 of q gains, then d/4 of k gains
+          const float4* src = et < d / 4 ? gq + et : gk + (et - d / 4);
+          const float4 g4 = a.qk_norm ? *src : make_float4(1.f, 1.f, 1.f, 1.f);
+          reinterpret_cast<float4*>(stg)[et] = g4;
+        }
+        qc.rope_rows = min(a.M, (stg_floats - 2 * d) / d);
+        if (l > 0) stage_rope();
         if (dv) {
           const size_t lo = (size_t)l * a.batch * a.Hkv * a.max_block * d;
           qc.kdst = a.blk_k + lo;
@@ -857,10 +863,49 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
       } else if (kind == PH_O || kind == PH_DOWN) {
         gam = kind == PH_O ? a.norms[l].mlp_norm : (l + 1 < a.L ? a.norms[l + 1].attn_norm : a.final_norm);
-        const int n = (last_tile - first_tile + 1) * 128;
-        if (n <= stg_floats) {
-          for (int i = et; i < n; i += 128) stg[i] = gam[(size_t)first_tile * 128 + i];
+        const int n4 = (last_tile - first_tile + 1) * 32;  // float4 of gains
+        if (n4 * 4 <= stg_floats) {
+          const float4* src = reinterpret_cast<const float4*>(gam + (size_t)first_tile * 128);
+          for (int b0 = 0; b0 < n4; b0 += 128 * 4) {
+            float4 buf[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = b0 + et + 128 * k;
+              buf[k] = i < n4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = b0 + et + 128 * k;
+              if (i < n4) reinterpret_cast<float4*>(stg)[i] = buf[k];
+            }
+          }
           gam_staged = true;
+        }
+      }
+      if (!acquire_phase(dep)) {
+        ok = false;
+        break;
+      }
+      if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E0);
+      if (kind == PH_QKV && l == 0) stage_rope();  // written by EMBED in this launch
+      if (kind == PH_QKV || kind == PH_GU || kind == PH_LM) {
+        // rstd of every token row from the D/128 per-tile sums of squares: thread (row m,
+        // quarter q) adds every fourth partial (its loads all in flight at once), then the
+        // four quarters are added in a fixed order
+        const int np = D / 128;
+        for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+          const int m = m0 + (et & 31), q = et >> 5;
+          float s = 0.f;
+          if (m < a.M) {
+#pragma unroll 8
+            for (int pp = q; pp < np; pp += 4) s += __ldcg(a.ss + (size_t)pp * a.ss_ld + m);
+          }
+          epi[et] = s;
+          named_bar_sync(1, 128);
+          if (q == 0 && m < a.Mt)
+            rstd_s[m] = m < a.M ? rsqrtf((((epi[et] + epi[32 + et]) + epi[64 + et]) + epi[96 + et]) / (float)D + a.eps)
+                                : 0.f;
+          named_bar_sync(1, 128);
         }
       }
       named_bar_sync(1, 128);

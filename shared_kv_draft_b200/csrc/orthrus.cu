@@ -823,6 +823,10 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
       const uint32_t box[4] = {64, 64, 2, 2};
       ok = ok && map_nd(P->lmap_mut(l, M_WGU4), lp.w_gu, 4, dims, strides, box);
     }
+    // the forward kernel reads norm gains as 16-byte vectors
+    auto a16 = [](const void* q) { return q != nullptr && ((uintptr_t)q & 15u) == 0; };
+    ok = ok && a16(lp.attn_norm) && a16(lp.mlp_norm) && a16(w->final_norm);
+    ok = ok && (!cfg->qk_norm || (a16(lp.q_norm) && a16(lp.k_norm) && a16(lp.wd_q_norm) && a16(lp.wd_k_norm)));
     LayerNorms& ln = P->norms_host()[l];
     ln.attn_norm = lp.attn_norm;
     ln.mlp_norm = lp.mlp_norm;
