@@ -515,11 +515,11 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
     }
   }
   if (m < m_valid) {
-    const int bb = m / a.Q, i = m - bb * a.Q;
+    const int bb = a.nb == 1 ? 0 : m / a.Q, i = m - bb * a.Q;  // (runtime divides cost ~100 cycles each)
     __nv_bfloat16* dst = nullptr;
     if (kind == 0) {
-      const int G = a.H / a.Hkv;
-      const int kvh = hh / G, g = hh - kvh * G;
+      const int G = a.G;
+      const int kvh = (G & (G - 1)) == 0 ? hh >> (31 - __clz(G)) : hh / G, g = hh - kvh * G;
       dst = a.qbuf + ((size_t)(bb * a.Hkv + kvh) * (a.Q * G) + i * G + g) * d;
     } else {
       const int kvh = hh - a.H - (kind == 2 ? a.Hkv : 0);
@@ -1260,25 +1260,45 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         if (nch > 1 && grow < g.rows_per_slot) {
           const int i = grow / a.G, gg = grow - i * a.G;
           const float2* ml = a.att_ml + (size_t)slot * kMaxChunks * 128 + r;
-          float mstar = -INFINITY;
-          for (int ch = 0; ch < nch; ++ch) mstar = fmaxf(mstar, __ldcg(ml + ch * 128).x);
-          float L = 0.f;
+          // online merge over batches of up to 8 chunks: a batch's (m, l) and O loads are all
+          // in flight together; the running maximum rescales the sums between batches
+          float mrun = -INFINITY, L = 0.f;
           float acc[per];
 #pragma unroll
           for (int e = 0; e < per; ++e) acc[e] = 0.f;
-          for (int ch = 0; ch < nch; ++ch) {
-            const float2 v = __ldcg(ml + ch * 128);
-            const float w = (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - mstar);
-            L += v.y * w;
-            const float4* po = reinterpret_cast<const float4*>(a.att_o) +
-                               (((size_t)slot * kMaxChunks + ch) * (d / 4) + sub * (per / 4)) * 128 + r;
+          for (int c0 = 0; c0 < nch; c0 += 8) {
+            float2 mlb[8];
+            float4 ob[8][per / 4];
 #pragma unroll
-            for (int e = 0; e < per / 4; ++e) {
-              const float4 x = __ldcg(po + (size_t)e * 128);
-              acc[4 * e] += w * x.x;
-              acc[4 * e + 1] += w * x.y;
-              acc[4 * e + 2] += w * x.z;
-              acc[4 * e + 3] += w * x.w;
+            for (int k = 0; k < 8; ++k) {
+              const bool in = c0 + k < nch;
+              mlb[k] = in ? __ldcg(ml + (c0 + k) * 128) : make_float2(-INFINITY, 0.f);
+              const float4* po = reinterpret_cast<const float4*>(a.att_o) +
+                                 (((size_t)slot * kMaxChunks + (in ? c0 + k : 0)) * (d / 4) + sub * (per / 4)) * 128 + r;
+#pragma unroll
+              for (int e = 0; e < per / 4; ++e) ob[k][e] = in ? __ldcg(po + (size_t)e * 128) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            float mb = mrun;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mb = fmaxf(mb, mlb[k].x);
+            if (mb != -INFINITY) {
+              const float sc = mrun == -INFINITY ? 0.f : fast_exp2(mrun - mb);
+              L *= sc;
+#pragma unroll
+              for (int e = 0; e < per; ++e) acc[e] *= sc;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float w = mlb[k].x == -INFINITY ? 0.f : fast_exp2(mlb[k].x - mb);
+                L += w * mlb[k].y;
+#pragma unroll
+                for (int e = 0; e < per / 4; ++e) {
+                  acc[4 * e] += w * ob[k][e].x;
+                  acc[4 * e + 1] += w * ob[k][e].y;
+                  acc[4 * e + 2] += w * ob[k][e].z;
+                  acc[4 * e + 3] += w * ob[k][e].w;
+                }
+              }
+              mrun = mb;
             }
           }
           const float inv = L > 0.f ? __fdividef(1.f, L) : 0.f;
