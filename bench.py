@@ -175,13 +175,21 @@ def run_ours(args, wl, rank, world, local_rank):
     m.prefill(tok, [P], pending)
 
     # greedy AR stream on the GPU (verify with K = 0); the timed run must reproduce it
+    # (also the plain-AR baseline: one token per forward through the same kernel, timed with CUDA events)
     stream_dev = i32(need)
     ar1, acc1 = i32(B, 1), i32(B)
     stream_dev[0] = pending[0]
+    ar_e0, ar_e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ar_w = min(3, need - 1)
     for j in range(1, need):
+        if j == ar_w + 1:
+            ar_e0.record()
         m.verify_block(pending, None, 0, ar1)
         m.accept_commit(pending, None, ar1, 0, acc1, stream_dev[j:j + 1])
+    ar_e1.record()
     torch.cuda.synchronize(dev)
+    ar_tokens = need - 1 - ar_w
+    ar_ms = ar_e0.elapsed_time(ar_e1) if ar_tokens > 0 else float("nan")
     if m.read_status() != 0:
         raise RuntimeError(f"device status {m.read_status()} while building the greedy stream")
     stream = stream_dev.cpu().numpy()
@@ -342,6 +350,7 @@ def run_ours(args, wl, rank, world, local_rank):
         "h2d": B * K * 4, "d2h": B * 4 + B * (K + 1) * 4, "hbm_peak": hbm_peak, "tf_peak": tf_peak,
         "peak_src": peak_src, "t_gen": t_gen, "weights": w, "stream": stream, "accepts": acc,
         "mean_committed": float(np.mean(acc[W:] + 1)), "cap": cap, "n_mean": n0 + int(np.sum(acc[W:] + 1)) // 2,
+        "ar_ms": ar_ms, "ar_tokens": ar_tokens,
     }
     return res
 
@@ -492,6 +501,14 @@ def main():
         "e2e": {"value": round(r["tokens"] / (r["e2e_ms"] * 1e-3), 2), "unit": "tok/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
     }
+    if r["ar_tokens"] > 0:
+        # plain greedy AR (one verify forward with K = 0 plus the commit per token) through the
+        # same kernels, on the same model and prompt: the like-for-like baseline of the speedup
+        ar_tps = r["ar_tokens"] / (r["ar_ms"] * 1e-3)
+        line["ar_baseline"] = {"value": round(ar_tps, 2), "unit": "tok/s", "tokens": r["ar_tokens"],
+                               "ms_per_token": round(r["ar_ms"] / r["ar_tokens"], 4),
+                               "speedup": round(value / ar_tps, 3),
+                               "path": "orthrus_verify_block(K=0) + orthrus_accept_commit per token"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores = oracle_step_time(wl["shape"], r["weights"], wl["K"], int(round(wl["mean_accept"])),
                                         r["stream"])

@@ -1169,8 +1169,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             uint32_t pk[16];
 #pragma unroll
             for (int tt = 0; tt < 32; tt += 2) {
-              const float p0 = (c0 + tt < nv) ? fast_exp2(sv[tt] * a.scale_log2 - m_new) : 0.f;
-              const float p1 = (c0 + tt + 1 < nv) ? fast_exp2(sv[tt + 1] * a.scale_log2 - m_new) : 0.f;
+              // masked keys get exp2(-inf) = 0: the select is on the argument, so no branch
+              // surrounds the (asm) exponential and the 32 of them can overlap
+              const float p0 = fast_exp2(c0 + tt < nv ? sv[tt] * a.scale_log2 - m_new : -INFINITY);
+              const float p1 = fast_exp2(c0 + tt + 1 < nv ? sv[tt + 1] * a.scale_log2 - m_new : -INFINITY);
               sum0 += p0;
               sum1 += p1;
               __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
