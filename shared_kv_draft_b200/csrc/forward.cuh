@@ -926,10 +926,11 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       };
       // partial slot of contributor cc to tile t: its first or its last segment
       auto part_slot = [&](int cc, int t) { return 2 * cc + (ust_s[cc] / kc == t ? 0 : 1); };
-      // next (up to) four non-empty contributors from cc on, in k order
+      // next (up to) two non-empty contributors from cc on, in k order (two per round: four
+      // rounds' worth of prefetched partials cost registers the rest of the kernel needs)
       auto gather4 = [&](int& cc, int c_hi, int& s0, int& s1, int& s2, int& s3, int t) {
         s0 = s1 = s2 = s3 = -1;
-        for (int q = 0; q < 4 && cc <= c_hi; ++cc) {
+        for (int q = 0; q < 2 && cc <= c_hi; ++cc) {
           if (ust_s[cc + 1] > ust_s[cc]) {
             const int sl = part_slot(cc, t);
             if (q == 0) s0 = sl;
@@ -940,9 +941,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           }
         }
       };
-      auto load4 = [&](float4 (&x)[4][8], int s0, int s1, int s2, int s3, int m0) {
+      auto load4 = [&](float4 (&x)[2][8], int s0, int s1, int s2, int s3, int m0) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           const int sl = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
           const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
                              (size_t)(m0 >> 2) * 128 + row;
@@ -952,9 +953,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       };
-      auto add4 = [&](float* v, const float4 (&x)[4][8]) {
+      auto add4 = [&](float* v, const float4 (&x)[2][8]) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)  // fixed k order within and across rounds
+        for (int q = 0; q < 2; ++q)  // fixed k order within and across rounds
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             v[4 * q4] += x[q][q4].x;
@@ -1057,7 +1058,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         int cc0 = c_lo + 1, s0, s1, s2, s3;
         gather4(cc0, c_hi, s0, s1, s2, s3, t);
-        float4 x[4][8];
+        float4 x[2][8];
         load4(x, s0, s1, s2, s3, 0);
         if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
           ok = false;
