@@ -1060,6 +1060,17 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         gather4(cc0, c_hi, s0, s1, s2, s3, t);
         float4 x[2][8];
         load4(x, s0, s1, s2, s3, 0);
+        // a second token group (the 33rd row of a K = 32 verify block) is usually one float4
+        // row: the same contributors' row 8 is loaded now too
+        float4 x2[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int sl = q == 0 ? s0 : s1;
+          x2[q] = (sl >= 0 && m_valid > 32)
+                      ? ld_f4_hint(reinterpret_cast<const float4*>(a.partial + (size_t)sl * (128 * 128)) + 8 * 128 + row,
+                                   pol_drop)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
           ok = false;
           break;
@@ -1071,6 +1082,28 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           int cc = c_lo + 1;
           if (m0 == 0) {
             add4(v, x);
+            cc = cc0;
+          } else if (m0 == 32) {
+            // the first round's contributors: row 8 prefetched, rows 9.. (tokens 36..) loaded here
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int sl = q == 0 ? s0 : s1;
+              const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
+                                 8 * 128 + row;
+              v[0] += x2[q].x;
+              v[1] += x2[q].y;
+              v[2] += x2[q].z;
+              v[3] += x2[q].w;
+#pragma unroll
+              for (int q4 = 1; q4 < 8; ++q4)
+                if (sl >= 0 && 32 + 4 * q4 < m_valid) {
+                  const float4 y = ld_f4_hint(pp + (size_t)q4 * 128, pol_drop);
+                  v[4 * q4] += y.x;
+                  v[4 * q4 + 1] += y.y;
+                  v[4 * q4 + 2] += y.z;
+                  v[4 * q4 + 3] += y.w;
+                }
+            }
             cc = cc0;
           }
           while (cc <= c_hi) {
