@@ -248,3 +248,53 @@ def test_batched_ragged_prefill_and_step():
         g, vl = o.verify_block(st, t["draft"][b].cpu().tolist())
         check_logits(t["vlog"][b].cpu().numpy(), vl, stats)
         check_tokens(t["ar"][b].cpu().tolist(), vl, stats)
+
+
+
+def test_large_batch_per_op_path_matches_oracle():
+    """Batch 16 with K = 8: 144 verify rows exceed the persistent kernel's 128, so draft and
+    verify run through the per-op kernels. Every sequence's draft and verify logits and
+    argmaxes match the oracle run on that sequence alone, and the accept/commit that
+    follows is consistent with the drafts and the AR argmax (bit-exact)."""
+    shape = synth.TINY_QK
+    K, B = 8, 16
+    rng = np.random.default_rng(77)
+    lens = rng.integers(5, 60, size=B).tolist()
+    cap = 80
+    w, dev = make_pair(shape, K, max(lens), cap, seed=12, batch=B)
+    o = Oracle(shape, w, capacity=cap)
+    toks = np.zeros((B, max(lens)), dtype=np.int32)
+    for b, L in enumerate(lens):
+        toks[b, :L] = synth.make_prompt(shape, L, 300 + b)
+    t = gpu_tensors(B, K, shape.vocab)
+    dev.prefill(torch.from_numpy(toks).cuda(), lens, t["pending"])
+    pend = t["pending"].cpu().numpy().copy()
+    dev.draft_block(t["pending"], K, t["draft"], t["dlog"])
+    dev.verify_block(t["pending"], t["draft"], K, t["ar"], t["vlog"])
+    dev.accept_commit(t["pending"], t["draft"], t["ar"], K, t["acc"], t["com"])
+    torch.cuda.synchronize()
+    assert dev.read_status() == 0
+    stats = Stats()
+    drafts, ar = t["draft"].cpu().numpy(), t["ar"].cpu().numpy()
+    acc, com = t["acc"].cpu().numpy(), t["com"].cpu().numpy()
+    new_lens, new_pend = dev.lens.cpu().numpy(), t["pending"].cpu().numpy()
+    for b, L in enumerate(lens):
+        st = o.new_state()
+        o.prefill(st, toks[b, :L])
+        last = o.forward(o.new_state(), toks[b, :L], "verify", last_only=True)
+        st.y = check_tokens([int(pend[b])], last, stats)[0]
+        _, dl = o.draft_block(st, K)
+        check_logits(t["dlog"][b].cpu().numpy(), dl, stats)
+        check_tokens(drafts[b].tolist(), dl, stats)
+        _, vl = o.verify_block(st, drafts[b].tolist())
+        check_logits(t["vlog"][b].cpu().numpy(), vl, stats)
+        check_tokens(ar[b].tolist(), vl, stats)
+        # the consensus on the GPU's own drafts and AR argmax, bit-exact
+        a = 0
+        while a < K and drafts[b, a] == ar[b, a]:
+            a += 1
+        assert acc[b] == a, (b, acc[b], a)
+        assert com[b, :a].tolist() == drafts[b, :a].tolist() and com[b, a] == ar[b, a], b
+        assert (com[b, a + 1:] == -1).all(), b
+        assert new_lens[b] == L + a + 1 and new_pend[b] == ar[b, a], b
+    print(stats)
