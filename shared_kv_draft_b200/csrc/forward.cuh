@@ -734,8 +734,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
   };
   // outputs of a completion unit written -> count it (the barrier orders the other
   // threads' stores before thread 0's release, which is cumulative)
-  auto signal = [&](int p) {
-    fence_proxy_async_global();
+  auto signal = [&](int p, bool async_readers = true) {
+    // the generic-proxy writes reach later TMA reads: proxy fence first (not needed when
+    // every reader uses plain loads)
+    if (async_readers) fence_proxy_async_global();
     named_bar_sync(1, 128);
     if (et == 0) red_release_gpu_add(a.phase_cnt + p, 1);
   };
@@ -928,23 +930,21 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
       auto part_slot = [&](int cc, int t) { return 2 * cc + (ust_s[cc] / kc == t ? 0 : 1); };
       // next (up to) two non-empty contributors from cc on, in k order (two per round: four
       // rounds' worth of prefetched partials cost registers the rest of the kernel needs)
-      auto gather4 = [&](int& cc, int c_hi, int& s0, int& s1, int& s2, int& s3, int t) {
-        s0 = s1 = s2 = s3 = -1;
+      auto gather2 = [&](int& cc, int c_hi, int& s0, int& s1, int t) {
+        s0 = s1 = -1;
         for (int q = 0; q < 2 && cc <= c_hi; ++cc) {
           if (ust_s[cc + 1] > ust_s[cc]) {
             const int sl = part_slot(cc, t);
             if (q == 0) s0 = sl;
-            else if (q == 1) s1 = sl;
-            else if (q == 2) s2 = sl;
-            else s3 = sl;
+            else s1 = sl;
             ++q;
           }
         }
       };
-      auto load4 = [&](float4 (&x)[2][8], int s0, int s1, int s2, int s3, int m0) {
+      auto load2 = [&](float4 (&x)[2][8], int s0, int s1, int m0) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          const int sl = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
+          const int sl = q == 0 ? s0 : s1;
           const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
                              (size_t)(m0 >> 2) * 128 + row;
 #pragma unroll
@@ -953,7 +953,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       };
-      auto add4 = [&](float* v, const float4 (&x)[2][8]) {
+      auto add2 = [&](float* v, const float4 (&x)[2][8]) {
 #pragma unroll
         for (int q = 0; q < 2; ++q)  // fixed k order within and across rounds
 #pragma unroll
@@ -1056,10 +1056,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           ok = false;
           break;
         }
-        int cc0 = c_lo + 1, s0, s1, s2, s3;
-        gather4(cc0, c_hi, s0, s1, s2, s3, t);
+        int cc0 = c_lo + 1, s0, s1;
+        gather2(cc0, c_hi, s0, s1, t);
         float4 x[2][8];
-        load4(x, s0, s1, s2, s3, 0);
+        load2(x, s0, s1, 0);
         // a second token group (the 33rd row of a K = 32 verify block) is usually one float4
         // row: the same contributors' row 8 is loaded now too
         float4 x2[2];
@@ -1081,7 +1081,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
           int cc = c_lo + 1;
           if (m0 == 0) {
-            add4(v, x);
+            add2(v, x);
             cc = cc0;
           } else if (m0 == 32) {
             // the first round's contributors: row 8 prefetched, rows 9.. (tokens 36..) loaded here
@@ -1107,9 +1107,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             cc = cc0;
           }
           while (cc <= c_hi) {
-            gather4(cc, c_hi, s0, s1, s2, s3, t);
-            load4(x, s0, s1, s2, s3, m0);
-            add4(v, x);
+            gather2(cc, c_hi, s0, s1, t);
+            load2(x, s0, s1, m0);
+            add2(v, x);
           }
           if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_LOAD);
           fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam_tile(nt), true);
@@ -1275,7 +1275,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           for (int e = 0; e < d; e += 4) __stcg(po + (size_t)(e / 4) * 128, make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
           __stcg(a.att_ml + pidx, make_float2(m_run, l_run));
         }
-        signal(p);
+        signal(p, t.n_chunks == 1);  // partials are read by the merge with plain loads
       }
       if (et == 0) tl_mark<TL>(a, n_ph, p, TL_E1);
     } else if (kind == PH_COMBINE) {
