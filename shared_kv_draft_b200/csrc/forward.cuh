@@ -92,7 +92,7 @@ constexpr int kMaxStages = 16;
 constexpr int kMaxSlots = 256;        // attention (sequence, kv head, row tile) slots per launch
 constexpr int kMaxChunks = 34;        // key chunks per slot (32 cache chunks + draft block + slack)
 constexpr int kCombineRows = 16;      // rows per merge unit
-constexpr int kScratchBytes = 17408;  // P tile (16 KB) / epilogue staging (32 x 132 fp32), shared
+constexpr int kScratchBytes = 19584;  // P tile (16 KB) / epilogue staging (36 x 132 fp32 + sums), shared
 constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers
 
 struct LayerNorms {  // device-resident per-layer gains (fp32)
@@ -194,7 +194,7 @@ __host__ __device__ inline int fwd_phase_layer(int p) { return (p - 1) / kPhases
 // a whole attention unit, so it cannot live in the ring), the P tile / epilogue
 // staging, small per-CTA tables and the barriers.
 __host__ inline size_t fwd_fixed_smem(int d) {
-  return 1024 /*align*/ + (size_t)128 * d * 2 /*Q*/ + kScratchBytes + 128 * 8 /*red*/ + 128 * 4 /*rstd*/ +
+  return 1024 /*align*/ + (size_t)128 * d * 2 /*Q*/ + kScratchBytes + 144 * 8 /*red*/ + 128 * 4 /*rstd*/ +
          128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/ +
          kMaxGrid * 4 /*unit-range starts*/;
 }
@@ -362,30 +362,28 @@ __device__ __forceinline__ void st_bf16x16(__nv_bfloat16* dst, const float* x) {
   p[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// Residual epilogue of the O and down projections on 32 token rows [m0, m0+32)
-// of one 128-column tile: h += v; xg = bf16(h * gamma_next); sum of h^2 over the
-// tile's 128 columns per row -> ss[nt][m]. With h_in_v the old h is already part
-// of v (added by the contributor that holds the tile's last k-chunk, early in its
-// range, so no h load sits on the path). gam_t: the next norm's gains of this
-// tile's 128 columns (shared memory when staged). Uses epi[32 * kEpiStride + 128)
-// for the per-quarter sums.
-__device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
-                                                   int m_valid, const float* gam_t, float* epi, bool h_in_v) {
+// Scratch layout of the epilogues (floats): the 32-row staging tile [32][kEpiStride],
+// 128 per-quarter sums, then the second group's staging [4][kEpiStride] and its 16
+// per-quarter sums. The second group carries token rows [m0+32, m0+32+n2), n2 <= 4:
+// the 33rd row of a K = 32 verify block goes through the same call as the first 32.
+constexpr int kEpiQsum = 32 * kEpiStride;
+constexpr int kEpi2 = kEpiQsum + 128;
+constexpr int kEpi2Qsum = kEpi2 + 4 * kEpiStride;
+constexpr int kEpiFloats = kEpi2Qsum + 16;
+static_assert(kEpiFloats * 4 <= kScratchBytes, "epilogue scratch");
+
+// second-group token count of a call on rows [m0, ...): rows past m0+32 when the block ends
+// within 4 of them (else the caller runs a separate call per 32 rows)
+__device__ __forceinline__ int epi_group2(int m0, int m_valid) {
+  const int n = m_valid - m0 - 32;
+  return n > 0 && n <= 4 ? n : 0;
+}
+
+// one (token row, 32-column quarter) of the residual epilogue: h row -> global, xg = bf16(h * gamma)
+// -> global; returns the quarter's sum of squares
+__device__ __forceinline__ float resid_quarter(const FwdArgs& a, const float* src, int m, int nt, int qq, bool store,
+                                               const float* gam_t) {
   const int D = a.D;
-  if (h_in_v) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
-  } else {
-    float hv[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      hv[j] = m0 + j < m_valid ? __ldcg(a.h + (size_t)(m0 + j) * D + nt * 128 + row) : 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j] + hv[j];
-  }
-  named_bar_sync(1, 128);
-  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
-  const float* src = epi + j * kEpiStride + qq * 32;
   float y[32];
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -403,10 +401,8 @@ __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float
     s2 += y[i + 2] * y[i + 2];
     s3 += y[i + 3] * y[i + 3];
   }
-  float* qsum = epi + 32 * kEpiStride;
-  qsum[qq * 32 + j] = (s0 + s1) + (s2 + s3);
-  if (m0 + j < m_valid) {
-    float4* hp = reinterpret_cast<float4*>(a.h + (size_t)(m0 + j) * D + nt * 128 + qq * 32);
+  if (store) {
+    float4* hp = reinterpret_cast<float4*>(a.h + (size_t)m * D + nt * 128 + qq * 32);
 #pragma unroll
     for (int c = 0; c < 8; ++c) hp[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
     const float4* gq = reinterpret_cast<const float4*>(gam_t + qq * 32);
@@ -415,13 +411,59 @@ __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float
       const float4 g4 = gq[c];
       y[4 * c] *= g4.x, y[4 * c + 1] *= g4.y, y[4 * c + 2] *= g4.z, y[4 * c + 3] *= g4.w;
     }
-    __nv_bfloat16* xp = a.xg + (size_t)(m0 + j) * D + nt * 128 + qq * 32;
+    __nv_bfloat16* xp = a.xg + (size_t)m * D + nt * 128 + qq * 32;
     st_bf16x16(xp, y);
     st_bf16x16(xp + 16, y + 16);
   }
+  return (s0 + s1) + (s2 + s3);
+}
+
+// Residual epilogue of the O and down projections on token rows [m0, m0+32) (+ the second
+// group v2) of one 128-column tile: h += v; xg = bf16(h * gamma_next); sum of h^2 over the
+// tile's 128 columns per row -> ss[nt][m]. With h_in_v the old h is already part of v (added
+// by the contributor that holds the tile's last k-chunk, early in its range, so no h load
+// sits on the path). gam_t: the next norm's gains of this tile's 128 columns.
+__device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float* v, const float* v2, int row, int m0,
+                                                   int nt, int m_valid, const float* gam_t, float* epi, bool h_in_v) {
+  const int D = a.D;
+  const int n2 = v2 ? epi_group2(m0, m_valid) : 0;
+  if (h_in_v) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < n2) epi[kEpi2 + k * kEpiStride + row] = v2[k];
+  } else {
+    float hv[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      hv[j] = m0 + j < m_valid ? __ldcg(a.h + (size_t)(m0 + j) * D + nt * 128 + row) : 0.f;
+    float hv2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) hv2[k] = k < n2 ? __ldcg(a.h + (size_t)(m0 + 32 + k) * D + nt * 128 + row) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j] + hv[j];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < n2) epi[kEpi2 + k * kEpiStride + row] = v2[k] + hv2[k];
+  }
   named_bar_sync(1, 128);
-  if (t < 32 && m0 + t < m_valid)
-    a.ss[(size_t)nt * a.ss_ld + m0 + t] = ((qsum[t] + qsum[32 + t]) + qsum[64 + t]) + qsum[96 + t];
+  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
+  epi[kEpiQsum + qq * 32 + j] =
+      resid_quarter(a, epi + j * kEpiStride + qq * 32, m0 + j, nt, qq, m0 + j < m_valid, gam_t);
+  if (t < 4 * n2) {  // second group: thread = (row k, quarter q2)
+    const int k = t >> 2, q2 = t & 3;
+    epi[kEpi2Qsum + q2 * 4 + k] = resid_quarter(a, epi + kEpi2 + k * kEpiStride + q2 * 32, m0 + 32 + k, nt, q2, true, gam_t);
+  }
+  named_bar_sync(1, 128);
+  if (t < 32 && m0 + t < m_valid) {
+    const float* q = epi + kEpiQsum;
+    a.ss[(size_t)nt * a.ss_ld + m0 + t] = ((q[t] + q[32 + t]) + q[64 + t]) + q[96 + t];
+  } else if (t >= 32 && t < 32 + n2) {
+    const int k = t - 32;
+    const float* q = epi + kEpi2Qsum;
+    a.ss[(size_t)nt * a.ss_ld + m0 + 32 + k] = ((q[k] + q[4 + k]) + q[8 + k]) + q[12 + k];
+  }
 }
 
 // Per-phase state of the q/k/v projection epilogue: destination of the block's
@@ -436,25 +478,17 @@ struct QkvCtx {
   int rope_rows;
 };
 
-// q/k/v epilogue on 32 token rows [m0, m0+32) of one 128-row tile (one head at
-// d = 128, two at d = 64): per-head RMSNorm of q and k, rotate-half RoPE at the
-// row's absolute position, bf16 store of q (qbuf) and of k, v (cache slot len+i
-// in the verify view, block-scratch row i in the draft view). Thread = (token row
-// j, quarter qq): d/32 threads per head, each holding elements [16s, 16s+16) and
-// their RoPE partners [d/2 + 16s, d/2 + 16s + 16).
+// one (token row m, quarter qq) of the q/k/v epilogue; src = the row's staged 128 columns.
+// Every lane of the warp runs it (the head's sum of squares is two shuffles); lanes with
+// valid == false store nothing.
 template <int D_HEAD>
-__device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx& q, const float* v, int row, int m0,
-                                                 int nt, int m_valid, float* epi, const int* lens_s) {
+__device__ __forceinline__ void qkv_item(const FwdArgs& a, const QkvCtx& q, const float* src_row, int m, int nt,
+                                         int qq, bool valid, const int* lens_s) {
   constexpr int d = D_HEAD, half = d / 2, TPH = d / 32;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
-  named_bar_sync(1, 128);
-  const int t = threadIdx.x - 64, j = t >> 2, qq = t & 3;
   const int hl = qq / TPH, e0 = 16 * (qq % TPH);
-  const int m = m0 + j;
   const int hh = (nt * 128) / d + hl;  // head index in the fused q|k|v rows
   const int kind = hh < a.H ? 0 : (hh < a.H + a.Hkv ? 1 : 2);
-  const float* src = epi + j * kEpiStride + hl * d;
+  const float* src = src_row + hl * d;
   float x1[16], x2[16];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -506,7 +540,7 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
         rot(2 * c, f.x, f.y);
         rot(2 * c + 1, f.z, f.w);
       }
-    } else if (m < m_valid) {
+    } else if (valid) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float2 f = a.rope[(size_t)m * half + e0 + i];
@@ -514,7 +548,7 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
       }
     }
   }
-  if (m < m_valid) {
+  if (valid) {
     const int bb = a.nb == 1 ? 0 : m / a.Q, i = m - bb * a.Q;  // (runtime divides cost ~100 cycles each)
     __nv_bfloat16* dst = nullptr;
     if (kind == 0) {
@@ -532,32 +566,63 @@ __device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx&
       st_bf16x16(dst + half + e0, x2);
     }
   }
+}
+
+// q/k/v epilogue on token rows [m0, m0+32) (+ the second group v2) of one 128-row tile (one
+// head at d = 128, two at d = 64): per-head RMSNorm of q and k, rotate-half RoPE at the row's
+// absolute position, bf16 store of q (qbuf) and of k, v (cache slot len+i in the verify view,
+// block-scratch row i in the draft view). Thread = (token row j, quarter qq): d/32 threads per
+// head, each holding elements [16s, 16s+16) and their RoPE partners [d/2 + 16s, d/2 + 16s + 16).
+// The second group's (row, quarter) items run on the first warp.
+template <int D_HEAD>
+__device__ __forceinline__ void fwd_qkv_epilogue(const FwdArgs& a, const QkvCtx& q, const float* v, const float* v2,
+                                                 int row, int m0, int nt, int m_valid, float* epi, const int* lens_s) {
+  const int n2 = v2 ? epi_group2(m0, m_valid) : 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (k < n2) epi[kEpi2 + k * kEpiStride + row] = v2[k];
+  named_bar_sync(1, 128);
+  const int t = threadIdx.x - 64, j = t >> 2, qq = t & 3;
+  qkv_item<D_HEAD>(a, q, epi + j * kEpiStride, m0 + j, nt, qq, m0 + j < m_valid, lens_s);
+  if (n2 > 0 && t < 32) {  // warp-uniform
+    const int k = min(j, 3);
+    qkv_item<D_HEAD>(a, q, epi + kEpi2 + k * kEpiStride, m0 + 32 + k, nt, qq, j < n2, lens_s);
+  }
   named_bar_sync(1, 128);
 }
 
 // SwiGLU epilogue of the gate/up projection on 32 token rows [m0, m0+32) of one
 // tile: rows 0..63 are the gate rows of features nt*64.., rows 64..127 the matching
 // up rows; act = silu(gate) * up in bf16. Thread = (token row, 16 features).
-__device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
-                                                    int m_valid, float* epi) {
+// one (token row, 16 features) of the SwiGLU epilogue; src = the row's staged columns
+__device__ __forceinline__ void swiglu_item(const FwdArgs& a, const float* src, int m, int nt, int qq) {
+  float y[16];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float4 g4 = *reinterpret_cast<const float4*>(src + 4 * c);
+    const float4 u4 = *reinterpret_cast<const float4*>(src + 64 + 4 * c);
+    const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)  // fast reciprocal: an IEEE divide branches per element
+      y[4 * c + i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * u[i];
+  }
+  st_bf16x16(a.act + (size_t)m * a.F + nt * 64 + 16 * qq, y);
+}
+
+__device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const float* v, const float* v2, int row, int m0,
+                                                    int nt, int m_valid, float* epi) {
+  const int n2 = v2 ? epi_group2(m0, m_valid) : 0;
 #pragma unroll
   for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (k < n2) epi[kEpi2 + k * kEpiStride + row] = v2[k];
   named_bar_sync(1, 128);
   const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
-  if (m0 + j < m_valid) {
-    const float* src = epi + j * kEpiStride + 16 * qq;
-    float y[16];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float4 g4 = *reinterpret_cast<const float4*>(src + 4 * c);
-      const float4 u4 = *reinterpret_cast<const float4*>(src + 64 + 4 * c);
-      const float g[4] = {g4.x, g4.y, g4.z, g4.w}, u[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)  // fast reciprocal: an IEEE divide branches per element
-        y[4 * c + i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * u[i];
-    }
-    st_bf16x16(a.act + (size_t)(m0 + j) * a.F + nt * 64 + 16 * qq, y);
-  }
+  if (m0 + j < m_valid) swiglu_item(a, epi + j * kEpiStride + 16 * qq, m0 + j, nt, qq);
+  if (t < 4 * n2) swiglu_item(a, epi + kEpi2 + (t >> 2) * kEpiStride + 16 * (t & 3), m0 + 32 + (t >> 2), nt, t & 3);
   named_bar_sync(1, 128);
 }
 
@@ -565,48 +630,64 @@ __device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const floa
 // vocabulary tile: optional fp32 logits, NaN check, and the running argmax key of
 // each token row. Thread = (token row, 32 vocabulary rows): the max over its 32
 // keys, then over the four quarters, then one atomic per token row.
-__device__ __forceinline__ void fwd_argmax_epilogue(const FwdArgs& a, const float* v, int row, int m0, int nt,
-                                                    int m_valid, float* epi, unsigned long long* red) {
+// one (token row m, 32 vocabulary rows) of the LM head: logits (optional), NaN check, key max
+__device__ __forceinline__ unsigned long long argmax_item(const FwdArgs& a, const float* src, int m, int nt, int qq) {
+  float y[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
-  named_bar_sync(1, 128);
-  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
-  const int m = m0 + j;
+  for (int c = 0; c < 8; ++c) {
+    const float4 f4 = *reinterpret_cast<const float4*>(src + 4 * c);
+    y[4 * c] = f4.x, y[4 * c + 1] = f4.y, y[4 * c + 2] = f4.z, y[4 * c + 3] = f4.w;
+  }
+  const uint32_t col0 = nt * 128 + qq * 32;  // vocabulary index of y[0]
   unsigned long long best = 0ull;
-  if (m < m_valid) {
-    const float* src = epi + j * kEpiStride + qq * 32;
-    float y[32];
+  bool bad = false;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float4 f4 = *reinterpret_cast<const float4*>(src + 4 * c);
-      y[4 * c] = f4.x, y[4 * c + 1] = f4.y, y[4 * c + 2] = f4.z, y[4 * c + 3] = f4.w;
-    }
-    const uint32_t col0 = nt * 128 + qq * 32;  // vocabulary index of y[0]
-    bool bad = false;
+  for (int i = 0; i < 32; ++i) {
+    const bool nan = isnan(y[i]);
+    bad |= nan;
+    best = ull_max(best, nan ? 0ull : argmax_key(y[i], col0 + i));
+  }
+  if (bad) set_status(a.status, ORTHRUS_ERR_NAN);
+  if (a.logits) {
+    float* lp = a.logits + (size_t)m * a.V + col0;
+    if ((a.V & 3) == 0) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const bool nan = isnan(y[i]);
-      bad |= nan;
-      best = ull_max(best, nan ? 0ull : argmax_key(y[i], col0 + i));
-    }
-    if (bad) set_status(a.status, ORTHRUS_ERR_NAN);
-    if (a.logits) {
-      float* lp = a.logits + (size_t)m * a.V + col0;
-      if ((a.V & 3) == 0) {
+      for (int c = 0; c < 8; ++c)
+        reinterpret_cast<float4*>(lp)[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+    } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          reinterpret_cast<float4*>(lp)[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) lp[i] = y[i];
-      }
+      for (int i = 0; i < 32; ++i) lp[i] = y[i];
     }
   }
-  red[qq * 32 + j] = best;
+  return best;
+}
+
+// Greedy head of the LM projection on token rows [m0, m0+32) (+ the second group v2) of one
+// 128-row vocabulary tile: thread = (token row, 32 vocabulary rows), the max over its keys,
+// then over the four quarters, then one atomic per token row. red: [128 + 16] keys.
+__device__ __forceinline__ void fwd_argmax_epilogue(const FwdArgs& a, const float* v, const float* v2, int row, int m0,
+                                                    int nt, int m_valid, float* epi, unsigned long long* red) {
+  const int n2 = v2 ? epi_group2(m0, m_valid) : 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) epi[j * kEpiStride + row] = v[j];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (k < n2) epi[kEpi2 + k * kEpiStride + row] = v2[k];
+  named_bar_sync(1, 128);
+  const int t = threadIdx.x - 64, j = t & 31, qq = t >> 5;
+  red[qq * 32 + j] = m0 + j < m_valid ? argmax_item(a, epi + j * kEpiStride + qq * 32, m0 + j, nt, qq) : 0ull;
+  if (t < 4 * n2) {  // second group: thread = (row k, quarter q2)
+    const int k = t >> 2, q2 = t & 3;
+    red[128 + q2 * 4 + k] = argmax_item(a, epi + kEpi2 + k * kEpiStride + q2 * 32, m0 + 32 + k, nt, q2);
+  }
   named_bar_sync(1, 128);
   if (t < 32 && m0 + t < m_valid) {
     const unsigned long long k = ull_max(ull_max(red[t], red[32 + t]), ull_max(red[64 + t], red[96 + t]));
     if (k != 0ull) atomicMax(a.amax + m0 + t, k);
+  } else if (t >= 32 && t < 32 + n2) {
+    const int k2 = t - 32;
+    const unsigned long long k = ull_max(ull_max(red[128 + k2], red[132 + k2]), ull_max(red[136 + k2], red[140 + k2]));
+    if (k != 0ull) atomicMax(a.amax + m0 + 32 + k2, k);
   }
 }
 
@@ -614,18 +695,22 @@ __device__ __forceinline__ void fwd_argmax_epilogue(const FwdArgs& a, const floa
 // normalised input first scale by rstd of the token row.
 template <int D_HEAD>
 __device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const QkvCtx& qc, const int* lens_s,
-                                             int epi_kind, float* v, int row, int m0, int nt, int m_valid, float* epi,
-                                             unsigned long long* red, const float* rstd_s, const float* gam_t,
-                                             bool h_in_v = false) {
+                                             int epi_kind, float* v, float* v2, int row, int m0, int nt, int m_valid,
+                                             float* epi, unsigned long long* red, const float* rstd_s,
+                                             const float* gam_t, bool h_in_v = false) {
   if (epi_kind == EPI_RESID) {
-    fwd_resid_epilogue(a, v, row, m0, nt, m_valid, gam_t, epi, h_in_v);
+    fwd_resid_epilogue(a, v, v2, row, m0, nt, m_valid, gam_t, epi, h_in_v);
     return;
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] *= rstd_s[m0 + j];
-  if (epi_kind == EPI_QKV) fwd_qkv_epilogue<D_HEAD>(a, qc, v, row, m0, nt, m_valid, epi, lens_s);
-  else if (epi_kind == EPI_SWIGLU) fwd_swiglu_epilogue(a, v, row, m0, nt, m_valid, epi);
-  else fwd_argmax_epilogue(a, v, row, m0, nt, m_valid, epi, red);
+  if (v2) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v2[k] *= rstd_s[m0 + 32 + k];
+  }
+  if (epi_kind == EPI_QKV) fwd_qkv_epilogue<D_HEAD>(a, qc, v, v2, row, m0, nt, m_valid, epi, lens_s);
+  else if (epi_kind == EPI_SWIGLU) fwd_swiglu_epilogue(a, v, v2, row, m0, nt, m_valid, epi);
+  else fwd_argmax_epilogue(a, v, v2, row, m0, nt, m_valid, epi, red);
 }
 
 }  // namespace orthrus
@@ -682,8 +767,10 @@ __device__ inline void fwd_finalize(const FwdArgs& a, int n_ph) {
   __threadfence();
 }
 
-// Epilogue warps (2-5) of the persistent forward kernel.
-template <int D_HEAD, bool TL>
+// Epilogue warps (2-5) of the persistent forward kernel. G2: the block has 33-36 token rows,
+// whose rows past 32 ride with the first epilogue call (a separate instantiation, so blocks of
+// at most 32 rows run without that code).
+template <int D_HEAD, bool TL, bool G2>
 __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeom& g, uint8_t* smem,
                                                   uint32_t stage_bytes, int S, uint8_t* scr,
                                                   unsigned long long* red, float* rstd_s, const int* lens_s,
@@ -916,6 +1003,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         return gam_staged ? stg + (t - first_tile) * 128 : gam + (size_t)t * 128;
       };
       const int m_valid = min(a.Mt, a.M);
+      const int n2 = G2 ? epi_group2(0, m_valid) : 0;  // rows past 32 that ride with the first call
       // owner of unit uu = the CTA whose non-empty range holds it (largest c with start <= uu)
       auto owner = [&](int uu) {
         int lo = 0, hi = Gd - 1;
@@ -983,8 +1071,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_ACC);
           tc_fence_after();
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+            if (m0 == 32 && n2 > 0) break;  // rows 32.. went with the first call
             tmem_ld32(taddr + m0, v);
-            fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam_tile(nt));
+            float v2[4];
+            if (m0 == 0 && n2 > 0) tmem_ld4(taddr + 32, v2);
+            fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, m0 == 0 && n2 > 0 ? v2 : nullptr, row, m0, nt, m_valid,
+                                 epi, red, rstd_s, gam_tile(nt));
           }
           tc_fence_before();
           __syncwarp();
@@ -1078,10 +1170,23 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_ACC);
         tc_fence_after();
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
+          if (m0 == 32 && n2 > 0) break;  // rows 32.. went with the first call
+          const bool fuse = m0 == 0 && n2 > 0;
           tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
+          float v2[4];
+          if (fuse) tmem_ld4(taddr + 32, v2);
           int cc = c_lo + 1;
           if (m0 == 0) {
             add2(v, x);
+            if (fuse) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                v2[0] += x2[q].x;
+                v2[1] += x2[q].y;
+                v2[2] += x2[q].z;
+                v2[3] += x2[q].w;
+              }
+            }
             cc = cc0;
           } else if (m0 == 32) {
             // the first round's contributors: row 8 prefetched, rows 9.. (tokens 36..) loaded here
@@ -1109,10 +1214,25 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           while (cc <= c_hi) {
             gather2(cc, c_hi, s0, s1, t);
             load2(x, s0, s1, m0);
+            if (fuse) {
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const int sl = q == 0 ? s0 : s1;
+                if (sl >= 0) {
+                  const float4 y = ld_f4_hint(
+                      reinterpret_cast<const float4*>(a.partial + (size_t)sl * (128 * 128)) + 8 * 128 + row, pol_drop);
+                  v2[0] += y.x;
+                  v2[1] += y.y;
+                  v2[2] += y.z;
+                  v2[3] += y.w;
+                }
+              }
+            }
             add2(v, x);
           }
           if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_LOAD);
-          fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, row, m0, nt, m_valid, epi, red, rstd_s, gam_tile(nt), true);
+          fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, fuse ? v2 : nullptr, row, m0, nt, m_valid, epi, red, rstd_s,
+                               gam_tile(nt), true);
         }
         tc_fence_before();
         __syncwarp();
@@ -1358,7 +1478,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
 
 namespace orthrus {
 
-template <int D_HEAD, bool TL>
+template <int D_HEAD, bool TL, bool G2>
 __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_constant__ FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1370,7 +1490,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   uint8_t* sQ = smem + (size_t)S * stage_bytes;   // attention Q tile, d/64 blocks of 128 rows x 64
   uint8_t* scr = sQ + (size_t)128 * d * 2;         // P tile / epilogue staging
   unsigned long long* red = (unsigned long long*)(scr + kScratchBytes);
-  float* rstd_s = (float*)(red + 128);
+  float* rstd_s = (float*)(red + 144);
   int* lens_s = (int*)(rstd_s + 128);
   int* slot_pre = lens_s + 128;
   int* ust_s = slot_pre + kMaxSlots + 1;  // [grid + 1] unit-range starts of the current phase
@@ -1704,7 +1824,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
     }
   } else {
     // ======================= epilogue warps =======================
-    fwd_epilogue_role<D_HEAD, TL>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, ust_s, accf, acce, full,
+    fwd_epilogue_role<D_HEAD, TL, G2>(a, g, smem, stage_bytes, S, scr, red, rstd_s, lens_s, slot_pre, ust_s, accf, acce, full,
                               s_full, p_full, o_full, flag, tmem_base, tS, tO);
   }
 

@@ -415,6 +415,19 @@ bool persistent_ok(const Plan* P, int Q) {
   return persistent_enabled() && P->mega_slots > 0 && P->B * Q <= 128 && Q <= P->max_block + 1;
 }
 
+template <int D, bool TL, bool G2>
+cudaError_t launch_forward_inst(cudaLaunchConfig_t& cfg, const FwdArgs& a) {
+  static bool set = false;
+  if (!set) set = set_smem_attr(forward_kernel<D, TL, G2>, kSmemLimit);
+  return cudaLaunchKernelEx(&cfg, forward_kernel<D, TL, G2>, a);
+}
+
+template <int D>
+cudaError_t launch_forward_d(cudaLaunchConfig_t& cfg, const FwdArgs& a, bool tl, bool g2) {
+  if (tl) return g2 ? launch_forward_inst<D, true, true>(cfg, a) : launch_forward_inst<D, true, false>(cfg, a);
+  return g2 ? launch_forward_inst<D, false, true>(cfg, a) : launch_forward_inst<D, false, false>(cfg, a);
+}
+
 orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending, const int* draft, int* out_ids,
                               float* logits, bool accept, int K, int* pending_out, int* accept_len, int* committed,
                               cudaStream_t st) {
@@ -504,28 +517,11 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  // the timeline instantiation only while a timeline buffer is set (profiling)
-  if (c.head_dim == 128) {
-    if (a.tl) {
-      static bool set = false;
-      if (!set) set = set_smem_attr(forward_kernel<128, true>, kSmemLimit);
-      e = cudaLaunchKernelEx(&cfg, forward_kernel<128, true>, a);
-    } else {
-      static bool set = false;
-      if (!set) set = set_smem_attr(forward_kernel<128, false>, kSmemLimit);
-      e = cudaLaunchKernelEx(&cfg, forward_kernel<128, false>, a);
-    }
-  } else {
-    if (a.tl) {
-      static bool set = false;
-      if (!set) set = set_smem_attr(forward_kernel<64, true>, kSmemLimit);
-      e = cudaLaunchKernelEx(&cfg, forward_kernel<64, true>, a);
-    } else {
-      static bool set = false;
-      if (!set) set = set_smem_attr(forward_kernel<64, false>, kSmemLimit);
-      e = cudaLaunchKernelEx(&cfg, forward_kernel<64, false>, a);
-    }
-  }
+  // the timeline instantiation only while a timeline buffer is set (profiling); the G2 one for
+  // blocks of 33-36 token rows (a K = 32 verify block)
+  const bool g2 = a.M > 32 && a.M <= 36;
+  if (c.head_dim == 128) e = launch_forward_d<128>(cfg, a, a.tl != nullptr, g2);
+  else e = launch_forward_d<64>(cfg, a, a.tl != nullptr, g2);
   return e == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }
 

@@ -298,3 +298,39 @@ def test_large_batch_per_op_path_matches_oracle():
         assert (com[b, a + 1:] == -1).all(), b
         assert new_lens[b] == L + a + 1 and new_pend[b] == ar[b, a], b
     print(stats)
+
+
+@pytest.mark.parametrize("B,K", [(1, 33), (4, 8), (2, 17)], ids=["rows34", "rows36", "rows36_b2"])
+def test_token_rows_past_32_match_oracle(B, K):
+    """Verify blocks of 34-36 token rows: the projections' epilogues handle a second group
+    of token columns past the first 32 (the 33rd row of a K = 32 verify block). Draft and
+    verify logits and argmaxes of every sequence match the oracle."""
+    shape = synth.TINY_QK
+    rng = np.random.default_rng(90 + B)
+    lens = rng.integers(10, 40, size=B).tolist()
+    cap = 40 + K + 8
+    w, dev = make_pair(shape, K, max(lens), cap, seed=13 + B, batch=B)
+    o = Oracle(shape, w, capacity=cap)
+    toks = np.zeros((B, max(lens)), dtype=np.int32)
+    for b, L in enumerate(lens):
+        toks[b, :L] = synth.make_prompt(shape, L, 400 + b)
+    t = gpu_tensors(B, K, shape.vocab)
+    dev.prefill(torch.from_numpy(toks).cuda(), lens, t["pending"])
+    pend = t["pending"].cpu().numpy().copy()
+    dev.draft_block(t["pending"], K, t["draft"], t["dlog"])
+    dev.verify_block(t["pending"], t["draft"], K, t["ar"], t["vlog"])
+    torch.cuda.synchronize()
+    assert dev.read_status() == 0
+    stats = Stats()
+    drafts = t["draft"].cpu().numpy()
+    for b, L in enumerate(lens):
+        st = o.new_state()
+        o.prefill(st, toks[b, :L])
+        last = o.forward(o.new_state(), toks[b, :L], "verify", last_only=True)
+        st.y = check_tokens([int(pend[b])], last, stats)[0]
+        _, dl = o.draft_block(st, K)
+        check_logits(t["dlog"][b].cpu().numpy(), dl, stats)
+        check_tokens(drafts[b].tolist(), dl, stats)
+        _, vl = o.verify_block(st, drafts[b].tolist())
+        check_logits(t["vlog"][b].cpu().numpy(), vl, stats)
+        check_tokens(t["ar"][b].cpu().tolist(), vl, stats)
