@@ -29,6 +29,8 @@ Readings where the pages are silent (each is stated where it is used):
 * Draft module = its own q/k/v/o projections (and q/k norm gains) with the
   shapes of the base attention; norms, MLP and LM head are the frozen ones.
 * Accept: a = number of leading i with d_i == g_{i-1}; commit d_1..d_a, g_a.
+* 2-step draft (atlas "Surprising findings"): a second draft-view pass over
+  [y, d_1..d_{K-1}], the first pass's predictions in place of the masks.
 * Decoder layer (Qwen3 style): pre-RMSNorm attention with optional per-head
   q/k RMSNorm and rotate-half RoPE, SwiGLU MLP, untied LM head.
 * K/V are rounded to bfloat16 when stored (the model's cache dtype); weights
@@ -273,6 +275,28 @@ class Oracle:
         logits = self.forward(st, ids, "draft")
         return [argmax_checked(logits[i]) for i in range(K)], logits
 
+    def draft_refine(self, st: SeqState, drafts):
+        """Second denoising step of the draft view (atlas summary "Surprising findings":
+        the 2-step iterative variant the single-step projection is compared with).
+
+        The pages leave its mechanism open; the reading taken here is the plainest one:
+        the masks of the first step are replaced by that step's predictions, i.e. the
+        draft view runs again over [y, d_1..d_{K-1}] at positions n..n+K-1 (block row i
+        still predicts position n+1+i, so d_K has no input slot and is not read), and
+        the new argmaxes d'_1..d'_K replace the drafts."""
+        K = len(drafts)
+        ids = [st.y] + [int(t) for t in drafts[:K - 1]]
+        logits = self.forward(st, ids, "draft")
+        return [argmax_checked(logits[i]) for i in range(K)], logits
+
+    def draft_steps(self, st: SeqState, K: int, steps: int):
+        """``steps`` denoising steps of the draft view: the single-step block
+        projection (steps = 1) followed by steps - 1 refinements."""
+        drafts, logits = self.draft_block(st, K)
+        for _ in range(steps - 1):
+            drafts, logits = self.draft_refine(st, drafts)
+        return drafts, logits
+
     def verify_block(self, st: SeqState, drafts):
         """Verify view over [y, d_1..d_K]; g_j = argmax of block row j (j = 0..K)."""
         ids = [st.y] + [int(t) for t in drafts]
@@ -304,15 +328,16 @@ def greedy_ar(model: Oracle, prompt, n_tokens: int):
     return st.out[:n_tokens]
 
 
-def orthrus_generate(model: Oracle, prompt, n_tokens: int, K: int, drafter=None):
+def orthrus_generate(model: Oracle, prompt, n_tokens: int, K: int, drafter=None, draft_steps: int = 1):
     """The Orthrus loop. ``drafter(model, st, K)`` returns d_1..d_K; by default the
-    draft view's argmax. Returns (tokens[:n_tokens], accept lengths)."""
+    draft view's argmax after ``draft_steps`` denoising steps. Returns
+    (tokens[:n_tokens], accept lengths)."""
     st = model.new_state()
     model.prefill(st, prompt)
     accepts = []
     while len(st.out) < n_tokens:
         if drafter is None:
-            drafts, _ = model.draft_block(st, K)
+            drafts, _ = model.draft_steps(st, K, draft_steps)
         else:
             drafts = [int(t) for t in drafter(model, st, K)]
         g, _ = model.verify_block(st, drafts)
