@@ -344,7 +344,10 @@ def run_ours(args, wl, rank, world, local_rank):
     if not np.array_equal(h_acc.numpy()[W:, 0], accepts[W:total_steps]):
         raise RuntimeError("end-to-end pass: accept lengths differ from the planted schedule")
 
+    variants = measure_variants(m, orthrus, dev, wl, W, Ksteps, planted_dev, accepts, reset, pending, cap, rank)
+
     res = {
+        "variants": variants,
         "ms": ms, "tokens": tokens, "bytes": bytes_total, "roofline": roof, "kernels": kernels, "clocks": clocks,
         "launches": launches_per_step * Ksteps, "e2e_ms": e2e_ms,
         "h2d": B * K * 4, "d2h": B * 4 + B * (K + 1) * 4, "hbm_peak": hbm_peak, "tf_peak": tf_peak,
@@ -353,6 +356,95 @@ def run_ours(args, wl, rank, world, local_rank):
         "ar_ms": ar_ms, "ar_tokens": ar_tokens,
     }
     return res
+
+
+def measure_variants(m, orthrus, dev, wl, W, Ksteps, planted_dev, accepts, reset, pending, cap, rank):
+    """Two decoding variants on the same model, timed with CUDA events after W warm-up steps:
+    - the 2-step iterative draft (orthrus_decode_step_ex, draft_steps = 2) on the planted
+      drafts of the main run (accept lengths must match the schedule);
+    - sampling at T = 1 (orthrus_decode_step_sampled): drafts drawn from the draft view,
+      rejection-sampling consensus with seeded uniforms; acceptance is whatever these
+      random-weight views give. The per-kernel split of one sampled step comes from the
+      library's event trace."""
+    import torch
+
+    shape, B, P, K = wl["shape"], wl["batch"], wl["prompt"], wl["K"]
+    V = shape.vocab
+    i32 = lambda *s: torch.zeros(s, dtype=torch.int32, device=dev)
+    out = {}
+    n = min(Ksteps, 24)
+    acc, com = i32(W + n, B), i32(W + n, B, K + 1)
+    reset()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for t in range(W + n):
+        if t == W:
+            e0.record()
+        m.decode_step_ex(pending, K, 2, planted_dev[t], acc[t], com[t])
+    e1.record()
+    torch.cuda.synchronize(dev)
+    if m.read_status() != 0 or not np.array_equal(acc.cpu().numpy()[:, 0], accepts[:W + n]):
+        raise RuntimeError("2-step draft run: accept lengths differ from the planted schedule")
+    ms = e0.elapsed_time(e1)
+    tok = int(np.sum(accepts[W:W + n] + 1)) * B
+    out["two_step_draft"] = {"value": round(tok / (ms * 1e-3), 2), "unit": "tok/s", "steps": n,
+                             "ms_per_step": round(ms / n, 4), "forwards_per_step": 3,
+                             "path": "orthrus_decode_step_ex(draft_steps=2), planted drafts"}
+
+    # sampling at T = 1: at most (K + 1) tokens per step must fit the cache
+    T = 1.0
+    n = max(0, min(Ksteps, 24, (cap - P - K - 2) // (K + 1) - W))
+    if n == 0:
+        return out
+    rng = np.random.default_rng(3000 + rank)
+    ud = torch.from_numpy(rng.random((W + n, B, K), dtype=np.float32)).to(dev)
+    ua = torch.from_numpy(rng.random((W + n, B, K), dtype=np.float32)).to(dev)
+    uf = torch.from_numpy(rng.random((W + n, B), dtype=np.float32)).to(dev)
+    dl = torch.empty((B, K, V), dtype=torch.float32, device=dev)
+    vl = torch.empty((B, K + 1, V), dtype=torch.float32, device=dev)
+    acc, com = i32(W + n, B), i32(W + n, B, K + 1)
+    reset()
+    for t in range(W + n):
+        if t == W:
+            e0.record()
+        m.decode_step_sampled(pending, K, T, ud[t], ua[t], uf[t], dl, vl, acc[t], com[t])
+    e1.record()
+    torch.cuda.synchronize(dev)
+    if m.read_status() != 0:
+        raise RuntimeError(f"sampled run: device status {m.read_status()}")
+    ms = e0.elapsed_time(e1)
+    a = acc.cpu().numpy()[W:, :]
+    tok = int(np.sum(a + 1))
+    # per-kernel split of sampled steps (event trace, same steps replayed from the same state)
+    reset()
+    for t in range(W):
+        m.decode_step_sampled(pending, K, T, ud[t], ua[t], uf[t], dl, vl, acc[t], com[t])
+    n_tr = min(n, 4)
+    n_ev = n_tr * 12 + 8
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in events:
+        e.record()
+    torch.cuda.synchronize(dev)
+    handles = (C.c_void_p * n_ev)(*[e.cuda_event for e in events])
+    kinds = (C.c_int32 * n_ev)()
+    count = (C.c_int32 * 1)(0)
+    m.trace(handles, kinds, count)
+    for t in range(W, W + n_tr):
+        m.decode_step_sampled(pending, K, T, ud[t], ua[t], uf[t], dl, vl, acc[t], com[t])
+    m.trace(None, None, None)
+    torch.cuda.synchronize(dev)
+    split = {}
+    for i in range(count[0] - 1):
+        if kinds[i] == 11:
+            continue
+        name = orthrus.KIND_NAMES[kinds[i]]
+        split[name] = split.get(name, 0.0) + events[i].elapsed_time(events[i + 1]) / n_tr
+    out["sampled_t1"] = {"value": round(tok / (ms * 1e-3), 2), "unit": "tok/s", "steps": n, "temperature": T,
+                         "ms_per_step": round(ms / n, 4), "mean_accept": round(float(np.mean(a)), 3),
+                         "ms_per_step_by_kind": {k: round(v, 4) for k, v in split.items()},
+                         "path": "orthrus_decode_step_sampled (draft view + draws, verify view, "
+                                 "rejection-sampling consensus)",
+                         "note": "acceptance of random-weight views, not of a trained draft module"}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -509,6 +601,7 @@ def main():
                                "ms_per_token": round(r["ar_ms"] / r["ar_tokens"], 4),
                                "speedup": round(value / ar_tps, 3),
                                "path": "orthrus_verify_block(K=0) + orthrus_accept_commit per token"}
+    line.update(r["variants"])  # the 2-step draft and sampling at T = 1, outside the timed region
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_cpu, cores = oracle_step_time(wl["shape"], r["weights"], wl["K"], int(round(wl["mean_accept"])),
                                         r["stream"])

@@ -160,8 +160,9 @@ enum {
   ORTHRUS_KIND_ACCEPT = 9,     /* greedy consensus + KV commit                     */
   ORTHRUS_KIND_OTHER = 10,     /* poisoning, length updates, planted-draft copy    */
   ORTHRUS_KIND_END = 11,       /* marker after the last launch of a call          */
-  ORTHRUS_KIND_FORWARD = 12    /* persistent kernel: one whole draft or verify forward
+  ORTHRUS_KIND_FORWARD = 12,   /* persistent kernel: one whole draft or verify forward
                                   (and, in orthrus_decode_step, the consensus)     */
+  ORTHRUS_KIND_SAMPLE = 13     /* temperature sampling: categorical draws, row statistics */
 };
 
 /* Profiling hook. While set, every launch made by the calls below is preceded
@@ -234,6 +235,79 @@ orthrus_status orthrus_accept_commit(const void* plan, int32_t* pending, const i
  * committed [batch][K+1] as in orthrus_accept_commit. */
 orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K, const int32_t* planted,
                                    int32_t* accept_len, int32_t* committed, orthrus_stream stream);
+
+/* Second (and further) denoising step of the draft view: the 2-step iterative
+ * variant that the single-step block projection is compared with (atlas
+ * summary "Surprising findings"). The pages leave the mechanism open; this
+ * call takes the plainest reading: the draft view runs again over
+ * [pending, prev_draft[0..K-2]] at positions len..len+K-1 (the previous step's
+ * predictions in place of the masks; prev_draft[K-1] has no input slot and is
+ * not read) and writes the new argmaxes to draft (device int32 [batch][K]).
+ * draft may be the same buffer as prev_draft (ids are read before any is
+ * written). logits (nullable): fp32 [batch][K][vocab]. The cache is read only.
+ * Errors: ORTHRUS_ERR_ARG (NULL pointers, K outside [1, max_block]); a draft
+ * id outside [0, vocab) sets the device status ORTHRUS_ERR_ARG. */
+orthrus_status orthrus_draft_refine(const void* plan, const int32_t* pending, const int32_t* prev_draft, int32_t K,
+                                    int32_t* draft, float* logits, orthrus_stream stream);
+
+/* orthrus_decode_step with draft_steps (1..8) denoising steps of the draft
+ * view: one orthrus_draft_block, then draft_steps - 1 orthrus_draft_refine in
+ * place, then (planted, verify, consensus) as orthrus_decode_step, which is
+ * this call with draft_steps = 1. */
+orthrus_status orthrus_decode_step_ex(const void* plan, int32_t* pending, int32_t K, int32_t draft_steps,
+                                      const int32_t* planted, int32_t* accept_len, int32_t* committed,
+                                      orthrus_stream stream);
+
+/* ---- decoding at temperature T > 0 (rejection sampling) ----------------
+ * The pages name rejection sampling as the method at T > 0 and describe it
+ * only briefly (atlas summary "Limitations"). These calls implement standard
+ * speculative sampling (Leviathan et al. 2023; Chen et al. 2023) on the
+ * Orthrus block, with every random number an input uniform on [0, 1):
+ *   q_i = softmax(draft logits row i / T), i = 0..K-1; d_{i+1} ~ q_i;
+ *   p_j = softmax(verify logits row j / T), j = 0..K;
+ *   d_i accepted iff u_accept[i-1] * q_{i-1}(d_i) < p_{i-1}(d_i), in order up
+ *   to the first rejection (a = number accepted); the last committed token is
+ *   drawn with u_final from max(0, p_a - q_a) (normalised) if d_{a+1} was
+ *   rejected, else from p_K (the bonus token).
+ * The committed tokens are then distributed as sampling from the frozen model
+ * at temperature T. A categorical draw with the uniform v is the inverse CDF:
+ * the first index (in index order) with positive weight whose running sum
+ * exceeds v times the total, sums in fp32. */
+
+/* One draw per row: out[r] ~ softmax(logits[r] / temperature) with
+ * uniforms[r]. logits: device fp32 [rows][vocab] (4-byte alignment is
+ * enough); uniforms: device fp32 [rows]; out: device int32 [rows].
+ * 1 <= vocab <= 262144; temperature > 0 and finite. status (device int32,
+ * nullable): set to ORTHRUS_ERR_NAN (and out[r] = -1) when a row holds a NaN
+ * or +inf logit or only -inf. Errors: ORTHRUS_ERR_ARG. No plan needed. */
+orthrus_status orthrus_sample_tokens(const float* logits, int32_t rows, int32_t vocab, float temperature,
+                                     const float* uniforms, int32_t* out, int32_t* status, orthrus_stream stream);
+
+/* Rejection-sampling consensus and KV commit (the T > 0 counterpart of
+ * orthrus_accept_commit, with the same outputs and bookkeeping: committed[b] =
+ * d_1..d_a, last token, then -1; accept_len[b] = a; cache.len[b] += a + 1;
+ * pending[b] = last token). draft: device int32 [batch][K]; draft_logits:
+ * fp32 [batch][K][vocab] (the orthrus_draft_block logits the drafts were drawn
+ * from); verify_logits: fp32 [batch][K+1][vocab] (orthrus_verify_block's);
+ * u_accept: fp32 [batch][K]; u_final: fp32 [batch]. K = 0 draws one token
+ * from p_0: plain sampled AR decoding (draft, draft_logits, u_accept may then
+ * be NULL). The row statistics go to the workspace. With the device status
+ * set (NaN logit, earlier error) nothing is committed and accept_len = -1.
+ * Errors: ORTHRUS_ERR_ARG. */
+orthrus_status orthrus_accept_sample(const void* plan, int32_t* pending, const int32_t* draft,
+                                     const float* draft_logits, const float* verify_logits, int32_t K,
+                                     float temperature, const float* u_accept, const float* u_final,
+                                     int32_t* accept_len, int32_t* committed, orthrus_stream stream);
+
+/* One Orthrus step at temperature T: draft view (logits to draft_logits),
+ * drafts drawn with u_draft (fp32 [batch][K]), verify view (logits to
+ * verify_logits), orthrus_accept_sample. draft_logits [batch][K][vocab] and
+ * verify_logits [batch][K+1][vocab] are caller-owned fp32 device buffers.
+ * Outputs as orthrus_accept_sample. */
+orthrus_status orthrus_decode_step_sampled(const void* plan, int32_t* pending, int32_t K, float temperature,
+                                           const float* u_draft, const float* u_accept, const float* u_final,
+                                           float* draft_logits, float* verify_logits, int32_t* accept_len,
+                                           int32_t* committed, orthrus_stream stream);
 
 /* ---- single kernels, exposed for parity tests and microbenchmarks ------ */
 

@@ -113,7 +113,7 @@ struct FwdArgs {
                              // so a row's softmax runs over the same absolute key chunks whatever
                              // the block size: verify rows equal the plain AR rows bit for bit
   const int* pending;        // [nb]
-  const int* draft_ids;      // [nb][Q-1] (verify)
+  const int* draft_ids;      // verify: [nb][Q-1]; draft: nullable [nb][Q], the previous drafts
   int* len;                  // [batch] (read; the fused accept advances it)
   const __nv_bfloat16* embed;
   const float* final_norm;
@@ -854,7 +854,8 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         const int bb = m / a.Q, i = m - bb * a.Q;
         int id;
         if (i == 0) id = a.pending[bb];
-        else id = a.view == VIEW_DRAFT ? a.mask_id : a.draft_ids[bb * (a.Q - 1) + i - 1];
+        else if (a.view == VIEW_VERIFY) id = a.draft_ids[bb * (a.Q - 1) + i - 1];
+        else id = a.draft_ids ? a.draft_ids[bb * a.Q + i - 1] : a.mask_id;  // refinement: previous drafts
         if (id < 0 || id >= a.V) {
           if (et == 0) set_status(a.status, ORTHRUS_ERR_ARG);
           id = 0;

@@ -15,6 +15,7 @@
 #include "forward.cuh"
 #include "gemm.cuh"
 #include "orthrus.h"
+#include "sampling.cuh"
 #include "small.cuh"
 
 using namespace orthrus;
@@ -145,6 +146,7 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // plan
 // ---------------------------------------------------------------------------
 constexpr uint64_t kPlanMagic = 0x4F52544852555331ull;  // "ORTHRUS1"
+constexpr int kMaxDraftSteps = 8;  // denoising steps of the draft view per decode step
 
 struct LayerPtrs {
   const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
@@ -168,6 +170,7 @@ struct alignas(64) Plan {
   float2* rope;
   unsigned long long* amax;
   int *draft_ids, *ar_ids;
+  float2* samp;  // per-row (max, normaliser) of the sampled consensus: [B * (2 max_block + 1)]
   float* gemm_part;
   int* gemm_cnt;
   float* att_o;
@@ -251,7 +254,7 @@ int attn_chunk_keys(int B, int Hkv, int row_tiles, int cap) {
 
 // workspace layout
 struct WsLayout {
-  size_t status, h, xn, qbuf, attn, act, rope, amax, draft_ids, ar_ids, gemm_part, gemm_cnt, att_o, att_ml, att_cnt,
+  size_t status, h, xn, qbuf, attn, act, rope, amax, draft_ids, ar_ids, samp, gemm_part, gemm_cnt, att_o, att_ml, att_cnt,
       blk_k, blk_v, dev_maps, dev_norms, phase_cnt, ss, fwd_att_o, fwd_att_ml, total;
   int chunk_keys, attn_slots, ss_ld, mega_slots;
 };
@@ -304,6 +307,7 @@ WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows_r
   w.amax = take((size_t)max_rows * 8);
   w.draft_ids = take((size_t)B * max_block * 4);
   w.ar_ids = take((size_t)B * (max_block + 1) * 4);
+  w.samp = take((size_t)B * (2 * max_block + 1) * 8);
   w.gemm_part = take((size_t)2 * sms * 128 * 128 * 4);
   w.gemm_cnt = take((size_t)gemm_counter_count(c, max_rows) * 4);
   w.att_o = take((size_t)w.attn_slots * 128 * d * 4);
@@ -760,6 +764,7 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->amax = (unsigned long long*)(base + wl.amax);
   P->draft_ids = (int*)(base + wl.draft_ids);
   P->ar_ids = (int*)(base + wl.ar_ids);
+  P->samp = (float2*)(base + wl.samp);
   P->gemm_part = (float*)(base + wl.gemm_part);
   P->gemm_cnt = (int*)(base + wl.gemm_cnt);
   P->att_o = (float*)(base + wl.att_o);
@@ -999,12 +1004,34 @@ orthrus_status orthrus_accept_commit(const void* plan, int32_t* pending, const i
   return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ERR_CUDA;
 }
 
-orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K, const int32_t* planted,
-                                   int32_t* accept_len, int32_t* committed, orthrus_stream stream) {
+orthrus_status orthrus_draft_refine(const void* plan, const int32_t* pending, const int32_t* prev_draft, int32_t K,
+                                    int32_t* draft, float* logits, orthrus_stream stream) {
   const Plan* P = plan_cast(plan);
-  if (!P || !pending || !accept_len || !committed || K < 1 || K > P->max_block) return ORTHRUS_ERR_ARG;
+  if (!P || !pending || !prev_draft || !draft || K < 1 || K > P->max_block) return ORTHRUS_ERR_ARG;
+  orthrus_status s;
+  if (persistent_ok(P, K)) {
+    mark(P, ORTHRUS_KIND_FORWARD, (cudaStream_t)stream);
+    s = launch_forward(P, VIEW_DRAFT, K, pending, prev_draft, draft, logits, false, 0, nullptr, nullptr, nullptr,
+                       (cudaStream_t)stream);
+  } else {
+    s = forward(P, BLOCK_DRAFT, 0, P->B, K, pending, prev_draft, nullptr, 0, 0, true, false, draft, logits,
+                (cudaStream_t)stream);
+  }
+  mark(P, ORTHRUS_KIND_END, (cudaStream_t)stream);
+  return s;
+}
+
+orthrus_status orthrus_decode_step_ex(const void* plan, int32_t* pending, int32_t K, int32_t draft_steps,
+                                      const int32_t* planted, int32_t* accept_len, int32_t* committed,
+                                      orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !accept_len || !committed || K < 1 || K > P->max_block || draft_steps < 1 ||
+      draft_steps > kMaxDraftSteps)
+    return ORTHRUS_ERR_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   orthrus_status s = orthrus_draft_block(plan, pending, K, P->draft_ids, nullptr, stream);
+  for (int i = 1; s == ORTHRUS_OK && i < draft_steps; ++i)  // in place: the ids are read before any is written
+    s = orthrus_draft_refine(plan, pending, P->draft_ids, K, P->draft_ids, nullptr, stream);
   if (s != ORTHRUS_OK) return s;
   if (planted) mark(P, ORTHRUS_KIND_OTHER, st);
   if (planted && cudaMemcpyAsync(P->draft_ids, planted, sizeof(int) * P->B * K, cudaMemcpyDeviceToDevice, st) !=
@@ -1020,6 +1047,71 @@ orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K
   s = orthrus_verify_block(plan, pending, P->draft_ids, K, P->ar_ids, nullptr, stream);
   if (s != ORTHRUS_OK) return s;
   return orthrus_accept_commit(plan, pending, P->draft_ids, P->ar_ids, K, accept_len, committed, 0, stream);
+}
+
+orthrus_status orthrus_decode_step(const void* plan, int32_t* pending, int32_t K, const int32_t* planted,
+                                   int32_t* accept_len, int32_t* committed, orthrus_stream stream) {
+  return orthrus_decode_step_ex(plan, pending, K, 1, planted, accept_len, committed, stream);
+}
+
+// ---- decoding at temperature T > 0 ------------------------------------------
+
+static bool temperature_ok(float t) { return t > 0.f && t < INFINITY; }
+
+orthrus_status orthrus_sample_tokens(const float* logits, int32_t rows, int32_t vocab, float temperature,
+                                     const float* uniforms, int32_t* out, int32_t* status, orthrus_stream stream) {
+  if (rows < 0 || vocab < 1 || vocab > kSampTile * kSampMaxTiles || !temperature_ok(temperature)) return ORTHRUS_ERR_ARG;
+  if (rows == 0) return ORTHRUS_OK;
+  if (!logits || !uniforms || !out) return ORTHRUS_ERR_ARG;
+  if (launch(sample_rows_kernel, dim3(rows), dim3(kSampThreads), 0, (cudaStream_t)stream, logits, (int)vocab,
+             1.f / temperature, uniforms, (int*)out, (int*)status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  return ORTHRUS_OK;
+}
+
+orthrus_status orthrus_accept_sample(const void* plan, int32_t* pending, const int32_t* draft,
+                                     const float* draft_logits, const float* verify_logits, int32_t K,
+                                     float temperature, const float* u_accept, const float* u_final,
+                                     int32_t* accept_len, int32_t* committed, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !verify_logits || !u_final || !accept_len || !committed || K < 0 || K > P->max_block ||
+      !temperature_ok(temperature) || P->cfg.vocab > kSampTile * kSampMaxTiles)
+    return ORTHRUS_ERR_ARG;
+  if (K > 0 && (!draft || !draft_logits || !u_accept)) return ORTHRUS_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = P->B, V = P->cfg.vocab;
+  const float inv_t = 1.f / temperature;
+  mark(P, ORTHRUS_KIND_SAMPLE, st);
+  if (launch(row_stats_kernel, dim3(B * (2 * K + 1)), dim3(kSampThreads), 0, st, draft_logits, B * K, verify_logits,
+             V, inv_t, P->samp, P->status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  mark(P, ORTHRUS_KIND_ACCEPT, st);
+  if (launch(accept_sample_kernel, dim3(B), dim3(kSampThreads), 0, st, (int*)pending, (const int*)draft, draft_logits,
+             verify_logits, (const float2*)P->samp, B, (int)K, V, inv_t, u_accept, u_final, (int*)accept_len,
+             (int*)committed, P->len, P->status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  mark(P, ORTHRUS_KIND_END, st);
+  return ORTHRUS_OK;
+}
+
+orthrus_status orthrus_decode_step_sampled(const void* plan, int32_t* pending, int32_t K, float temperature,
+                                           const float* u_draft, const float* u_accept, const float* u_final,
+                                           float* draft_logits, float* verify_logits, int32_t* accept_len,
+                                           int32_t* committed, orthrus_stream stream) {
+  const Plan* P = plan_cast(plan);
+  if (!P || !pending || !u_draft || !u_accept || !u_final || !draft_logits || !verify_logits || !accept_len ||
+      !committed || K < 1 || K > P->max_block || !temperature_ok(temperature))
+    return ORTHRUS_ERR_ARG;
+  orthrus_status s = orthrus_draft_block(plan, pending, K, P->draft_ids, draft_logits, stream);
+  if (s != ORTHRUS_OK) return s;
+  mark(P, ORTHRUS_KIND_SAMPLE, (cudaStream_t)stream);
+  s = orthrus_sample_tokens(draft_logits, P->B * K, P->cfg.vocab, temperature, u_draft, P->draft_ids, P->status,
+                            stream);
+  if (s != ORTHRUS_OK) return s;
+  s = orthrus_verify_block(plan, pending, P->draft_ids, K, P->ar_ids, verify_logits, stream);
+  if (s != ORTHRUS_OK) return s;
+  return orthrus_accept_sample(plan, pending, P->draft_ids, draft_logits, verify_logits, K, temperature, u_accept,
+                               u_final, accept_len, committed, stream);
 }
 
 // ---- single kernels -------------------------------------------------------

@@ -12,7 +12,7 @@ struct EmbedArgs {
   int kind, nb, b0, Q, D, d, V, mask_id, cap;
   double theta;
   const int* pending;   // [batch]            (draft, verify)
-  const int* draft;     // [nb][Q-1]          (verify)
+  const int* draft;     // verify: [nb][Q-1]; draft: nullable [nb][Q], previous drafts
   const int* tokens;    // prefill: tokens[b * tok_stride + tok_off + i]
   int tok_stride, tok_off;
   const int* len;       // [batch]
@@ -23,7 +23,8 @@ struct EmbedArgs {
 };
 
 // Block row m = bb*Q + i holds sequence b0+bb at position len[b]+i:
-//   draft:   ids [y, MASK x (Q-1)]
+//   draft:   ids [y, MASK x (Q-1)], or [y, d_1 .. d_{Q-1}] of the previous drafts
+//            (draft [nb][Q]) in a refinement step
 //   verify:  ids [y, d_1 .. d_{Q-1}]
 //   prefill: prompt tokens
 __global__ void embed_kernel(const EmbedArgs a) {
@@ -35,7 +36,8 @@ __global__ void embed_kernel(const EmbedArgs a) {
   int id;
   if (a.kind == BLOCK_PREFILL) id = a.tokens[(size_t)b * a.tok_stride + a.tok_off + i];
   else if (i == 0) id = a.pending[b];
-  else id = (a.kind == BLOCK_DRAFT) ? a.mask_id : a.draft[bb * (a.Q - 1) + (i - 1)];
+  else if (a.kind != BLOCK_DRAFT) id = a.draft[bb * (a.Q - 1) + (i - 1)];
+  else id = a.draft ? a.draft[bb * a.Q + (i - 1)] : a.mask_id;  // refinement: previous drafts
   if (id < 0 || id >= a.V) {
     if (threadIdx.x == 0) set_status(a.status, ORTHRUS_ERR_ARG);
     id = 0;

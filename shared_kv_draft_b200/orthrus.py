@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liborthrus.so")
 
 KIND_NAMES = ["embed", "rmsnorm", "gemm_qkv", "attention", "gemm_o", "gemm_gate_up", "gemm_down", "lm_head",
-              "argmax", "accept", "other", "end", "forward"]
+              "argmax", "accept", "other", "end", "forward", "sample"]
 
 OK, ERR_ARG, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_NAN, ERR_UNSUPPORTED, ERR_WORKSPACE = range(8)
 STATUS_NAMES = {0: "OK", 1: "ARG", 2: "CAPACITY", 3: "CUDA", 4: "TIMEOUT", 5: "NAN", 6: "UNSUPPORTED",
@@ -73,6 +73,11 @@ SIGNATURES = [
     ("orthrus_verify_block", _I32, [_VP, _VP, _VP, _I32, _VP, _VP, _VP]),
     ("orthrus_accept_commit", _I32, [_VP, _VP, _VP, _VP, _I32, _VP, _VP, _I32, _VP]),
     ("orthrus_decode_step", _I32, [_VP, _VP, _I32, _VP, _VP, _VP, _VP]),
+    ("orthrus_draft_refine", _I32, [_VP, _VP, _VP, _I32, _VP, _VP, _VP]),
+    ("orthrus_decode_step_ex", _I32, [_VP, _VP, _I32, _I32, _VP, _VP, _VP, _VP]),
+    ("orthrus_sample_tokens", _I32, [_VP, _I32, _I32, _F, _VP, _VP, _VP, _VP]),
+    ("orthrus_accept_sample", _I32, [_VP, _VP, _VP, _VP, _VP, _I32, _F, _VP, _VP, _VP, _VP, _VP]),
+    ("orthrus_decode_step_sampled", _I32, [_VP, _VP, _I32, _F, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     ("orthrus_attention_workspace_bytes", _SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
     ("orthrus_attention", _I32, [_VP, _VP, _VP, _VP, _VP, _VP, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _VP,
                                  _VP, _SZ, _VP, _VP]),
@@ -173,6 +178,14 @@ def linear_noalloc(X, W, Y, status=None, stream=None):
     _check("orthrus_linear_noalloc", code)
 
 
+def sample_tokens(logits, temperature, uniforms, out, status=None, stream=None):
+    """out[r] ~ softmax(logits[r] / temperature) drawn with uniforms[r] (device fp32 [rows][vocab])."""
+    rows, vocab = logits.shape
+    code = load().orthrus_sample_tokens(_ptr(logits), rows, vocab, float(temperature), _ptr(uniforms), _ptr(out),
+                                        _ptr(status), _stream(stream))
+    _check("orthrus_sample_tokens", code)
+
+
 def linear_workspace_bytes(M, N, Kd) -> int:
     return load().orthrus_linear_workspace_bytes(M, N, Kd)
 
@@ -258,6 +271,31 @@ class DeviceModel:
         _check("orthrus_decode_step",
                load().orthrus_decode_step(self.plan, _ptr(pending), K, _ptr(planted), _ptr(accept_len),
                                           _ptr(committed), _stream(stream)))
+
+    def draft_refine(self, pending, prev_draft, K, draft, logits=None, stream=None):
+        _check("orthrus_draft_refine",
+               load().orthrus_draft_refine(self.plan, _ptr(pending), _ptr(prev_draft), K, _ptr(draft), _ptr(logits),
+                                           _stream(stream)))
+
+    def decode_step_ex(self, pending, K, draft_steps, planted, accept_len, committed, stream=None):
+        _check("orthrus_decode_step_ex",
+               load().orthrus_decode_step_ex(self.plan, _ptr(pending), K, draft_steps, _ptr(planted),
+                                             _ptr(accept_len), _ptr(committed), _stream(stream)))
+
+    def accept_sample(self, pending, draft, draft_logits, verify_logits, K, temperature, u_accept, u_final,
+                      accept_len, committed, stream=None):
+        _check("orthrus_accept_sample",
+               load().orthrus_accept_sample(self.plan, _ptr(pending), _ptr(draft), _ptr(draft_logits),
+                                            _ptr(verify_logits), K, float(temperature), _ptr(u_accept),
+                                            _ptr(u_final), _ptr(accept_len), _ptr(committed), _stream(stream)))
+
+    def decode_step_sampled(self, pending, K, temperature, u_draft, u_accept, u_final, draft_logits, verify_logits,
+                            accept_len, committed, stream=None):
+        _check("orthrus_decode_step_sampled",
+               load().orthrus_decode_step_sampled(self.plan, _ptr(pending), K, float(temperature), _ptr(u_draft),
+                                                  _ptr(u_accept), _ptr(u_final), _ptr(draft_logits),
+                                                  _ptr(verify_logits), _ptr(accept_len), _ptr(committed),
+                                                  _stream(stream)))
 
     def clear_status(self, stream=None):
         _check("orthrus_clear_status", load().orthrus_clear_status(self.plan, _stream(stream)))

@@ -77,3 +77,21 @@ def test_plan_init_rejects_nulls(lib):
     cache = orthrus.Cache(None, None, None, 1, 64)
     code = lib.orthrus_plan_init(buf, n, C.byref(cfg), C.byref(w), C.byref(cache), 4, 5, None, 0, None)
     assert code == orthrus.ERR_ARG
+
+
+def test_refine_and_sampling_calls_check_arguments_on_the_host(lib):
+    nan, inf = float("nan"), float("inf")
+    assert lib.orthrus_draft_refine(None, None, None, 4, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_decode_step_ex(None, None, 4, 2, None, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_accept_sample(None, None, None, None, None, 4, 1.0, None, None, None, None,
+                                     None) == orthrus.ERR_ARG
+    assert lib.orthrus_decode_step_sampled(None, None, 4, 1.0, None, None, None, None, None, None, None,
+                                           None) == orthrus.ERR_ARG
+    # temperature must be positive and finite; 1 <= vocab <= 262144; rows >= 0
+    for t in (0.0, -1.0, nan, inf):
+        assert lib.orthrus_sample_tokens(None, 1, 1024, t, None, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_sample_tokens(None, 1, 0, 1.0, None, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_sample_tokens(None, 1, 262145, 1.0, None, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_sample_tokens(None, -1, 1024, 1.0, None, None, None, None) == orthrus.ERR_ARG
+    assert lib.orthrus_sample_tokens(None, 1, 1024, 1.0, None, None, None, None) == orthrus.ERR_ARG  # NULL buffers
+    assert lib.orthrus_sample_tokens(None, 0, 1024, 1.0, None, None, None, None) == orthrus.OK       # nothing to do
