@@ -170,7 +170,8 @@ struct alignas(64) Plan {
   float2* rope;
   unsigned long long* amax;
   int *draft_ids, *ar_ids;
-  float2* samp;  // per-row (max, normaliser) of the sampled consensus: [B * (2 max_block + 1)]
+  float2* samp;     // per-row (max, normaliser) of the sampling kernels: [B * (2 max_block + 1)]
+  float* samp_tot;  // per-row CDF tile totals: [B * max_block][kSampMaxTiles]
   float* gemm_part;
   int* gemm_cnt;
   float* att_o;
@@ -254,7 +255,7 @@ int attn_chunk_keys(int B, int Hkv, int row_tiles, int cap) {
 
 // workspace layout
 struct WsLayout {
-  size_t status, h, xn, qbuf, attn, act, rope, amax, draft_ids, ar_ids, samp, gemm_part, gemm_cnt, att_o, att_ml, att_cnt,
+  size_t status, h, xn, qbuf, attn, act, rope, amax, draft_ids, ar_ids, samp, samp_tot, gemm_part, gemm_cnt, att_o, att_ml, att_cnt,
       blk_k, blk_v, dev_maps, dev_norms, phase_cnt, ss, fwd_att_o, fwd_att_ml, total;
   int chunk_keys, attn_slots, ss_ld, mega_slots;
 };
@@ -308,6 +309,7 @@ WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows_r
   w.draft_ids = take((size_t)B * max_block * 4);
   w.ar_ids = take((size_t)B * (max_block + 1) * 4);
   w.samp = take((size_t)B * (2 * max_block + 1) * 8);
+  w.samp_tot = take((size_t)B * max_block * kSampMaxTiles * 4);
   w.gemm_part = take((size_t)2 * sms * 128 * 128 * 4);
   w.gemm_cnt = take((size_t)gemm_counter_count(c, max_rows) * 4);
   w.att_o = take((size_t)w.attn_slots * 128 * d * 4);
@@ -765,6 +767,7 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->draft_ids = (int*)(base + wl.draft_ids);
   P->ar_ids = (int*)(base + wl.ar_ids);
   P->samp = (float2*)(base + wl.samp);
+  P->samp_tot = (float*)(base + wl.samp_tot);
   P->gemm_part = (float*)(base + wl.gemm_part);
   P->gemm_cnt = (int*)(base + wl.gemm_cnt);
   P->att_o = (float*)(base + wl.att_o);
@@ -1069,6 +1072,46 @@ orthrus_status orthrus_sample_tokens(const float* logits, int32_t rows, int32_t 
   return ORTHRUS_OK;
 }
 
+// The consensus of a sampled step: statistics of the verify rows (and of the draft rows unless
+// the draws already computed them), tile totals of the last token's weights, draw and commit.
+static orthrus_status sampled_consensus(const Plan* P, int32_t* pending, const int32_t* draft, const float* dl,
+                                        const float* vl, int K, float temperature, const float* u_accept,
+                                        const float* u_final, int32_t* accept_len, int32_t* committed,
+                                        bool draft_stats_ready, cudaStream_t st) {
+  const int B = P->B, V = P->cfg.vocab;
+  const float inv_t = 1.f / temperature;
+  mark(P, ORTHRUS_KIND_SAMPLE, st);
+  const int skip = draft_stats_ready ? B * K : 0;  // rows whose statistics are already in place
+  if (launch(row_stats_kernel, dim3(B * (2 * K + 1) - skip), dim3(kSampThreads), 0, st, dl, B * K - skip, vl, V,
+             inv_t, P->samp + skip, P->status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  ConsensusArgs c;
+  c.pending = (int*)pending;
+  c.draft = (const int*)draft;
+  c.dl = dl;
+  c.vl = vl;
+  c.stats = P->samp;
+  c.tot = P->samp_tot;
+  c.u_acc = u_accept;
+  c.u_fin = u_final;
+  c.accept_len = (int*)accept_len;
+  c.committed = (int*)committed;
+  c.len = P->len;
+  c.status = P->status;
+  c.B = B;
+  c.K = K;
+  c.V = V;
+  c.inv_t = inv_t;
+  const int nt = (V + kSampTile - 1) / kSampTile;
+  mark(P, ORTHRUS_KIND_ACCEPT, st);
+  if (launch(consensus_totals_kernel, dim3(B, (nt + kTotTiles - 1) / kTotTiles), dim3(kTotThreads), 0, st, c) !=
+      cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  if (launch(consensus_select_kernel, dim3(B), dim3(kTotThreads), 0, st, c) != cudaSuccess) return ORTHRUS_ERR_CUDA;
+  mark(P, ORTHRUS_KIND_END, st);
+  return ORTHRUS_OK;
+}
+
 orthrus_status orthrus_accept_sample(const void* plan, int32_t* pending, const int32_t* draft,
                                      const float* draft_logits, const float* verify_logits, int32_t K,
                                      float temperature, const float* u_accept, const float* u_final,
@@ -1078,20 +1121,8 @@ orthrus_status orthrus_accept_sample(const void* plan, int32_t* pending, const i
       !temperature_ok(temperature) || P->cfg.vocab > kSampTile * kSampMaxTiles)
     return ORTHRUS_ERR_ARG;
   if (K > 0 && (!draft || !draft_logits || !u_accept)) return ORTHRUS_ERR_ARG;
-  cudaStream_t st = (cudaStream_t)stream;
-  const int B = P->B, V = P->cfg.vocab;
-  const float inv_t = 1.f / temperature;
-  mark(P, ORTHRUS_KIND_SAMPLE, st);
-  if (launch(row_stats_kernel, dim3(B * (2 * K + 1)), dim3(kSampThreads), 0, st, draft_logits, B * K, verify_logits,
-             V, inv_t, P->samp, P->status) != cudaSuccess)
-    return ORTHRUS_ERR_CUDA;
-  mark(P, ORTHRUS_KIND_ACCEPT, st);
-  if (launch(accept_sample_kernel, dim3(B), dim3(kSampThreads), 0, st, (int*)pending, (const int*)draft, draft_logits,
-             verify_logits, (const float2*)P->samp, B, (int)K, V, inv_t, u_accept, u_final, (int*)accept_len,
-             (int*)committed, P->len, P->status) != cudaSuccess)
-    return ORTHRUS_ERR_CUDA;
-  mark(P, ORTHRUS_KIND_END, st);
-  return ORTHRUS_OK;
+  return sampled_consensus(P, pending, draft, draft_logits, verify_logits, K, temperature, u_accept, u_final,
+                           accept_len, committed, false, (cudaStream_t)stream);
 }
 
 orthrus_status orthrus_decode_step_sampled(const void* plan, int32_t* pending, int32_t K, float temperature,
@@ -1100,18 +1131,30 @@ orthrus_status orthrus_decode_step_sampled(const void* plan, int32_t* pending, i
                                            int32_t* committed, orthrus_stream stream) {
   const Plan* P = plan_cast(plan);
   if (!P || !pending || !u_draft || !u_accept || !u_final || !draft_logits || !verify_logits || !accept_len ||
-      !committed || K < 1 || K > P->max_block || !temperature_ok(temperature))
+      !committed || K < 1 || K > P->max_block || !temperature_ok(temperature) ||
+      P->cfg.vocab > kSampTile * kSampMaxTiles)
     return ORTHRUS_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
   orthrus_status s = orthrus_draft_block(plan, pending, K, P->draft_ids, draft_logits, stream);
   if (s != ORTHRUS_OK) return s;
-  mark(P, ORTHRUS_KIND_SAMPLE, (cudaStream_t)stream);
-  s = orthrus_sample_tokens(draft_logits, P->B * K, P->cfg.vocab, temperature, u_draft, P->draft_ids, P->status,
-                            stream);
-  if (s != ORTHRUS_OK) return s;
+  // the drafts: statistics of the draft rows, tile totals, draws (the indices orthrus_sample_tokens gives)
+  const int rows = P->B * K, V = P->cfg.vocab, nt = (V + kSampTile - 1) / kSampTile;
+  const float inv_t = 1.f / temperature;
+  mark(P, ORTHRUS_KIND_SAMPLE, st);
+  if (launch(row_stats_kernel, dim3(rows), dim3(kSampThreads), 0, st, (const float*)draft_logits, rows,
+             (const float*)nullptr, V, inv_t, P->samp, P->status) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  if (launch(draw_totals_kernel, dim3(rows, (nt + kTotTiles - 1) / kTotTiles), dim3(kTotThreads), 0, st,
+             (const float*)draft_logits, V, inv_t, (const float2*)P->samp, P->samp_tot) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  if (launch(draw_select_kernel, dim3(rows), dim3(32), 0, st, (const float*)draft_logits, V, inv_t,
+             (const float2*)P->samp, (const float*)P->samp_tot, u_draft, P->draft_ids) != cudaSuccess)
+    return ORTHRUS_ERR_CUDA;
+  mark(P, ORTHRUS_KIND_END, st);
   s = orthrus_verify_block(plan, pending, P->draft_ids, K, P->ar_ids, verify_logits, stream);
   if (s != ORTHRUS_OK) return s;
-  return orthrus_accept_sample(plan, pending, P->draft_ids, draft_logits, verify_logits, K, temperature, u_accept,
-                               u_final, accept_len, committed, stream);
+  return sampled_consensus(P, pending, P->draft_ids, draft_logits, verify_logits, K, temperature, u_accept, u_final,
+                           accept_len, committed, true, st);
 }
 
 // ---- single kernels -------------------------------------------------------
