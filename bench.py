@@ -45,11 +45,19 @@ KV_BYTES_PER_POSITION = None
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "forward_kernel_traffic.json")
 
 
+# CUDA sources that hold no code of the persistent forward kernel (its traffic record stays valid
+# when only these change)
+NOT_FORWARD_SOURCES = {"sampling.cuh"}
+
+
 def kernel_sources_sha256():
-    """sha256 over the CUDA sources of the library (file name + contents, sorted by path)."""
+    """sha256 over the CUDA sources the persistent forward kernel is built from (file name +
+    contents, sorted by path): every file of csrc/ except NOT_FORWARD_SOURCES."""
     csrc = os.path.join(ROOT, "shared_kv_draft_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.cu"))):
+        if os.path.basename(f) in NOT_FORWARD_SOURCES:
+            continue
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
