@@ -185,10 +185,14 @@ __device__ int sample_row(const W& w, int V, float v, SampleSmem& sm) {
 
 // One warp: the draw from the tile totals tot[0..nt) that tile_prepare gave for these weights.
 // The same fp32 operations as sample_row (running sums from 0 in tile order, target = v * total,
-// the rescan of the chosen tile), so the result is the same index.
+// the rescan of the chosen tile), so the result is the same index. The totals are first copied
+// to `stage` (shared memory, kSampMaxTiles floats) by the whole warp, so that lane 0's running
+// sums read shared memory instead of waiting on one global load per tile.
 template <class W>
-__device__ int select_from_totals(const W& w, int V, float v, const float* tot, int lane) {
+__device__ int select_from_totals(const W& w, int V, float v, const float* tot_global, float* tot, int lane) {
   const int nt = (V + kSampTile - 1) / kSampTile;
+  for (int s = lane; s < nt; s += 32) tot[s] = tot_global[s];
+  __syncwarp();
   int sel = -1, last = -1;
   float base = 0.f, target = 0.f;
   if (lane == 0) {
@@ -348,12 +352,13 @@ __global__ void __launch_bounds__(32) draw_select_kernel(const float* logits, in
                                                          const float* uniforms, int* out) {
   griddep_wait();
   griddep_launch();
+  __shared__ float stage[kSampMaxTiles];
   const int row = blockIdx.x, lane = threadIdx.x;
   const float m = stats[row].x;
   int r = -1;
   if (m == m)
     r = select_from_totals(TemperedWeight{logits + (size_t)row * V, m, inv_t}, V, uniforms[row],
-                           tot + (size_t)row * kSampMaxTiles, lane);
+                           tot + (size_t)row * kSampMaxTiles, stage, lane);
   if (lane == 0) out[row] = r;
 }
 
@@ -437,12 +442,13 @@ __global__ void __launch_bounds__(kTotThreads) consensus_select_kernel(const Con
   __shared__ SampleSmem sm;
   __shared__ unsigned masks[2];
   __shared__ int last_s;
+  __shared__ float stage[kSampMaxTiles];
   const int b = blockIdx.x, t = threadIdx.x, K = c.K;
   const int a = consensus_accept_len(c, b, masks);
   if (t < 32) {
     const float* tot = c.tot + (size_t)b * kSampMaxTiles;
-    const int r = a < K ? select_from_totals(residual_weight(c, b, a), c.V, c.u_fin[b], tot, t)
-                        : select_from_totals(verify_weight(c, b, a), c.V, c.u_fin[b], tot, t);
+    const int r = a < K ? select_from_totals(residual_weight(c, b, a), c.V, c.u_fin[b], tot, stage, t)
+                        : select_from_totals(verify_weight(c, b, a), c.V, c.u_fin[b], tot, stage, t);
     if (t == 0) last_s = r;
   }
   __syncthreads();
