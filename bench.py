@@ -79,6 +79,25 @@ def captured_traffic(kernel, algo_bytes):
     return round(algo_bytes * ratio)
 
 
+def rank_reduce(x, op, world, dev):
+    """x reduced over the ranks with op ("max", "min" or "sum"); x itself on a single rank.
+    Every rank must call it, in the same order (it is a collective)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op={"max": dist.ReduceOp.MAX, "min": dist.ReduceOp.MIN, "sum": dist.ReduceOp.SUM}[op])
+    return int(round(t.item())) if isinstance(x, int) else float(t.item())
+
+
+def raise_on_any_rank(err, world, dev):
+    """A collective every rank takes after its checks: all ranks raise if any rank found an
+    error, so that no rank is left waiting in a later collective."""
+    if rank_reduce(1 if err else 0, "max", world, dev):
+        raise RuntimeError(err or "another rank failed its checks")
+
+
 def shape_bytes(shape):
     """Weight bytes streamed by one forward and KV bytes per cached position (all layers)."""
     D, H, Hkv, d, F, V, L = (shape.d_model, shape.n_heads, shape.n_kv_heads, shape.head_dim, shape.d_ff, shape.vocab,
@@ -242,25 +261,23 @@ def run_ours(args, wl, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = rank_reduce(ev0.elapsed_time(ev1), "max", world, dev)
 
     # ---- checks: accept lengths as planted, committed stream == greedy stream -----------------
-    if m.read_status() != 0:
-        raise RuntimeError(f"device status {m.read_status()} after the timed run")
+    err = None
     acc = acc_all.cpu().numpy()[:, 0]
     com = com_all.cpu().numpy()[:, 0]
-    if not np.array_equal(acc, accepts[:total_steps]):
-        raise RuntimeError("accept lengths differ from the planted schedule")
     out = [int(stream[0])]
     for t in range(total_steps):
-        out.extend(int(x) for x in com[t, :acc[t] + 1])
-    if out != [int(x) for x in stream[:len(out)]]:
-        raise RuntimeError("committed stream differs from the greedy stream")
-    tokens = int(np.sum(acc[W:] + 1)) * world
+        out.extend(int(x) for x in com[t, :max(acc[t], 0) + 1])
+    if m.read_status() != 0:
+        err = f"device status {m.read_status()} after the timed run"
+    elif not np.array_equal(acc, accepts[:total_steps]):
+        err = "accept lengths differ from the planted schedule"
+    elif out != [int(x) for x in stream[:len(out)]]:
+        err = "committed stream differs from the greedy stream"
+    raise_on_any_rank(err, world, dev)
+    tokens = rank_reduce(int(np.sum(acc[W:] + 1)), "sum", world, dev)  # all ranks' committed tokens
     # algorithmic HBM bytes of the timed steps
     wbytes, kvpos = shape_bytes(shape)
     n0 = P + int(np.sum(acc[:W] + 1))
@@ -344,13 +361,9 @@ def run_ours(args, wl, rank, world, local_rank):
         h_com[t].copy_(com_all[t], non_blocking=True)
     e1.record()
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    if not np.array_equal(h_acc.numpy()[W:, 0], accepts[W:total_steps]):
-        raise RuntimeError("end-to-end pass: accept lengths differ from the planted schedule")
+    e2e_ms = rank_reduce(e0.elapsed_time(e1), "max", world, dev)
+    raise_on_any_rank(None if np.array_equal(h_acc.numpy()[W:, 0], accepts[W:total_steps])
+                      else "end-to-end pass: accept lengths differ from the planted schedule", world, dev)
 
     try:  # measured after the main line's numbers; a failure here must not cost the main line
         variants = measure_variants(m, orthrus, dev, wl, W, Ksteps, planted_dev, accepts, reset, pending, cap,
