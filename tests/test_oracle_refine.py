@@ -95,3 +95,44 @@ def test_draft_steps_counts_passes(monkeypatch):
     assert [v for v, _ in calls] == ["draft", "draft"]
     assert calls[0][1] == [st.y, m.s.mask_id, m.s.mask_id]
     assert calls[1][1] == [st.y] + first[:2]
+
+
+# ---- planted mistakes in the refinement -------------------------------------------------
+
+def refine_shifted(self, st, drafts):  # d_2..d_K in the slots instead of d_1..d_{K-1}
+    K = len(drafts)
+    logits = self.forward(st, [st.y] + [int(t) for t in drafts[1:K]], "draft")
+    return [int(torch.argmax(logits[i])) for i in range(K)], logits
+
+
+def refine_without_pending(self, st, drafts):  # the block starts at d_1: y dropped
+    K = len(drafts)
+    logits = self.forward(st, [int(t) for t in drafts[:K]], "draft")
+    return [int(torch.argmax(logits[i])) for i in range(K)], logits
+
+
+def refine_verify_view(self, st, drafts):  # the frozen causal view instead of the draft view
+    K = len(drafts)
+    saved = (st.n, [k.clone() for k in st.k], [v.clone() for v in st.v])
+    logits = self.forward(st, [st.y] + [int(t) for t in drafts[:K - 1]], "verify")
+    st.n, st.k, st.v = saved
+    return [int(torch.argmax(logits[i])) for i in range(K)], logits
+
+
+def brute_pin_holds(m, s, w):
+    prompt = [3, 1, 4, 1, 5, 9]
+    st = m.new_state()
+    m.prefill(st, prompt)
+    prev = [7, 2, 11, 0]
+    _, lg = m.draft_refine(st, prev)
+    ref = np.array(brute_run(s, w, prompt, [st.y, 7, 2, 11], True))
+    return bool(np.allclose(lg.numpy(), ref, rtol=1e-9, atol=1e-11))
+
+
+@pytest.mark.parametrize("mistake", [refine_shifted, refine_without_pending, refine_verify_view],
+                         ids=lambda f: f.__name__)
+def test_planted_refinement_mistake_is_caught(mistake, monkeypatch):
+    s, w, m = micro_model()
+    assert brute_pin_holds(m, s, w)
+    monkeypatch.setattr(om.Oracle, "draft_refine", mistake)
+    assert not brute_pin_holds(m, s, w)
