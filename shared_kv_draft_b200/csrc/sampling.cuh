@@ -24,9 +24,9 @@
 
 namespace orthrus {
 
-constexpr int kSampThreads = 512;  // row statistics and the plan-free draws: one CTA per row
-constexpr int kSampTile = 1024;       // elements of one CDF tile
-constexpr int kSampMaxTiles = 256;    // vocab <= 262144
+constexpr int kSampThreads = 512;   // row statistics and the plan-free draws: one CTA per row
+constexpr int kSampTile = 1024;     // elements of one CDF tile
+constexpr int kSampMaxTiles = 256;  // vocab <= 262144
 
 __device__ __forceinline__ float warp_incl_scan(float x, int lane) {
 #pragma unroll
