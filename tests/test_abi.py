@@ -95,3 +95,15 @@ def test_refine_and_sampling_calls_check_arguments_on_the_host(lib):
     assert lib.orthrus_sample_tokens(None, -1, 1024, 1.0, None, None, None, None) == orthrus.ERR_ARG
     assert lib.orthrus_sample_tokens(None, 1, 1024, 1.0, None, None, None, None) == orthrus.ERR_ARG  # NULL buffers
     assert lib.orthrus_sample_tokens(None, 0, 1024, 1.0, None, None, None, None) == orthrus.OK       # nothing to do
+
+
+def test_header_is_plain_c():
+    """include/orthrus.h is a C header: it compiles as C99 with no C++ or CUDA types."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    r = subprocess.run([gcc, "-std=c99", "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", "c",
+                        os.path.join(ROOT, "include", "orthrus.h")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
