@@ -107,3 +107,37 @@ def test_header_is_plain_c():
     r = subprocess.run([gcc, "-std=c99", "-fsyntax-only", "-Wall", "-Wextra", "-Werror", "-x", "c",
                         os.path.join(ROOT, "include", "orthrus.h")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def declared_prototypes():
+    """name -> list of parameter declarations, from include/orthrus.h."""
+    text = open(os.path.join(ROOT, "include", "orthrus.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(orthrus_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = [p.strip() for p in m.group(2).replace("\n", " ").split(",")]
+        out[m.group(1)] = [] if params == ["void"] else params
+    return out
+
+
+def ctype_of(param):
+    """The ctypes type a parameter declaration must be bound with."""
+    decl = re.sub(r"\s+", " ", param)
+    if "*" in decl or decl.startswith("orthrus_stream"):
+        return "pointer"
+    base = decl.rsplit(" ", 1)[0].replace("const ", "")
+    return {"int32_t": C.c_int32, "size_t": C.c_size_t, "float": C.c_float}[base]
+
+
+def test_binding_signatures_match_the_header():
+    protos = declared_prototypes()
+    assert set(protos) == set(declared_symbols())
+    for name, res, args in orthrus.SIGNATURES:
+        params = protos[name]
+        assert len(args) == len(params), (name, len(args), len(params))
+        for a, p in zip(args, params):
+            want = ctype_of(p)
+            if want == "pointer":
+                assert a is C.c_void_p or issubclass(a, C._Pointer), (name, p, a)
+            else:
+                assert a is want, (name, p, a)
