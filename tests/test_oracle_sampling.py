@@ -277,3 +277,29 @@ def test_planted_mistake_is_caught(mistake, monkeypatch):
     p0, q0, p1 = random_pair(1)
     got = first_token_distribution(p0, q0, p1, N=400)
     assert np.abs(got - p0).max() > 0.02
+
+
+def test_sampled_step_on_the_decoder_reduces_to_the_greedy_step_when_cold():
+    """The oracle's whole sampled step on a tiny decoder: at T -> 0 the draws are the
+    argmaxes and the consensus is the greedy one, so the step commits what the greedy step
+    commits; the cache bookkeeping is the greedy step's."""
+    import synth
+    from oracle import Oracle
+    from test_oracle_bruteforce import Micro
+    s = Micro()
+    w = synth.make_weights(s, 31, 32, std=0.3, gain_std=0.3, threads=1)
+    m = Oracle(s, w, capacity=64, rowwise=True)
+    rng = np.random.default_rng(8)
+    cold, greedy = m.new_state(), m.new_state()
+    prompt = [3, 1, 4, 1, 5, 9, 2, 6]
+    m.prefill(cold, prompt)
+    m.prefill(greedy, prompt)
+    K = 4
+    for _ in range(5):
+        ud, ua, uf = osamp.step_uniforms(rng, 1, K)
+        d_ref, _ = m.draft_block(greedy, K)
+        g, _ = m.verify_block(greedy, d_ref)
+        a_ref, toks_ref = m.accept_commit(greedy, d_ref, g)
+        drafts, a, toks = osamp.sampled_step(m, cold, K, 1e-4, ud[0], ua[0], float(uf[0]))
+        assert drafts == d_ref and a == a_ref and toks == toks_ref
+        assert cold.n == greedy.n and cold.y == greedy.y
