@@ -117,6 +117,28 @@ def attention(q: torch.Tensor, keys: torch.Tensor, vals: torch.Tensor, n_visible
     return out.reshape(Q, H * d)
 
 
+def attention_by_head(q: torch.Tensor, keys: torch.Tensor, vals: torch.Tensor, n_visible) -> torch.Tensor:
+    """The same grouped-query attention, one head at a time over all query rows:
+    scores of row i against keys [0, n_visible[i]) with the others masked to -inf, then
+    the softmax and the weighted sum of the values. Keys past max(n_visible) are never
+    read. Used when the rows need not be evaluated one at a time (long caches)."""
+    Q, H, d = q.shape
+    Hkv = keys.shape[0]
+    G = H // Hkv
+    nmax = int(max(n_visible)) if Q else 0
+    out = torch.empty((Q, H, d), dtype=F64)
+    mask = torch.arange(nmax)[None, :] < torch.as_tensor([int(x) for x in n_visible])[:, None]  # [Q, nmax]
+    scale = 1.0 / math.sqrt(d)
+    for h in range(H):
+        kv = h // G
+        s = (q[:, h] @ keys[kv, :nmax].T) * scale
+        s = s.masked_fill(~mask, -math.inf)
+        p = torch.exp(s - s.max(dim=1, keepdim=True).values)
+        p = p / p.sum(dim=1, keepdim=True)
+        out[:, h] = p @ vals[kv, :nmax]
+    return out.reshape(Q, H * d)
+
+
 def argmax_checked(logits_row: torch.Tensor) -> int:
     if torch.isnan(logits_row).any():
         raise FloatingPointError("NaN logit")
@@ -172,8 +194,10 @@ class Oracle:
     ``weights`` maps tensor names to uint16 bfloat16 bits (matrices) or float32
     gains, with the row layouts: w_qkv rows = q heads | k heads | v heads;
     w_gate_up rows = gate | up.
-    ``rowwise=True`` evaluates every linear layer one row at a time, so that a
-    row's result never depends on which other rows share the block.
+    ``rowwise=True`` evaluates every linear layer and the attention one row at a
+    time, so that a row's result never depends on which other rows share the block;
+    otherwise rows are evaluated together (a matrix product per layer, attention one
+    head at a time), which is faster and equal up to float64 rounding order.
     """
 
     def __init__(self, shape, weights: dict, capacity: int, rowwise: bool = False):
@@ -189,9 +213,11 @@ class Oracle:
 
     # -- state ------------------------------------------------------------
     def new_state(self) -> SeqState:
+        """Cache slots hold bf16 values (K and V are rounded to bf16 when stored), so they
+        are kept as bfloat16: lossless, and a quarter of the float64 footprint."""
         s = self.s
-        k = [torch.zeros((s.n_kv_heads, self.cap, s.head_dim), dtype=F64) for _ in range(s.n_layers)]
-        v = [torch.zeros((s.n_kv_heads, self.cap, s.head_dim), dtype=F64) for _ in range(s.n_layers)]
+        k = [torch.zeros((s.n_kv_heads, self.cap, s.head_dim), dtype=torch.bfloat16) for _ in range(s.n_layers)]
+        v = [torch.zeros((s.n_kv_heads, self.cap, s.head_dim), dtype=torch.bfloat16) for _ in range(s.n_layers)]
         return SeqState(k=k, v=v)
 
     # -- one forward over a block of positions n .. n+Q-1 -------------------
@@ -239,12 +265,12 @@ class Oracle:
             k = rope(k, pos, s.rope_theta)
             k = round_bf16(k)
             v = round_bf16(v)
-            keys = torch.cat([st.k[l][:, :n], k.permute(1, 0, 2)], dim=1)
-            vals = torch.cat([st.v[l][:, :n], v.permute(1, 0, 2)], dim=1)
-            if view == "verify":
-                st.k[l][:, n:n + Q] = k.permute(1, 0, 2)
-                st.v[l][:, n:n + Q] = v.permute(1, 0, 2)
-            o = attention(q, keys, vals, n_visible)
+            keys = torch.cat([st.k[l][:, :n].to(F64), k.permute(1, 0, 2)], dim=1)
+            vals = torch.cat([st.v[l][:, :n].to(F64), v.permute(1, 0, 2)], dim=1)
+            if view == "verify":  # bf16 values: stored exactly
+                st.k[l][:, n:n + Q] = k.permute(1, 0, 2).to(torch.bfloat16)
+                st.v[l][:, n:n + Q] = v.permute(1, 0, 2).to(torch.bfloat16)
+            o = attention(q, keys, vals, n_visible) if self.rowwise else attention_by_head(q, keys, vals, n_visible)
             if return_qkv:
                 trace.append({"q": q.clone(), "k": k.clone(), "v": v.clone(), "o": o.clone()})
             h = h + linear(o, w[p + pre + "o"], self.rowwise)

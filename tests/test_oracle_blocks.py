@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import attention, linear, rms_norm, rope, silu
+from oracle import attention, attention_by_head, linear, rms_norm, rope, silu
 
 F64 = torch.float64
 
@@ -31,9 +31,13 @@ def brute_attention(q, keys, vals, n_visible):
     return out
 
 
+ATTENTION_FORMS = [attention, attention_by_head]
+
+
+@pytest.mark.parametrize("attention", ATTENTION_FORMS, ids=["by_row", "by_head"])
 @pytest.mark.parametrize("H,Hkv", [(1, 1), (2, 1), (4, 2), (4, 1), (2, 2)])
 @pytest.mark.parametrize("mode", ["all", "causal"])
-def test_attention_matches_brute_force(H, Hkv, mode):
+def test_attention_matches_brute_force(H, Hkv, mode, attention):
     rng = np.random.default_rng(H * 10 + Hkv)
     d, n, Q = 4, 5, 3
     q = rng.standard_normal((Q, H, d))
@@ -45,7 +49,8 @@ def test_attention_matches_brute_force(H, Hkv, mode):
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
 
 
-def test_attention_special_cases():
+@pytest.mark.parametrize("attention", ATTENTION_FORMS, ids=["by_row", "by_head"])
+def test_attention_special_cases(attention):
     rng = np.random.default_rng(5)
     d = 8
     q = torch.tensor(rng.standard_normal((1, 2, d)))
@@ -70,7 +75,8 @@ def test_attention_special_cases():
     assert torch.equal(a, b)
 
 
-def test_gqa_group_reads_its_kv_head():
+@pytest.mark.parametrize("attention", ATTENTION_FORMS, ids=["by_row", "by_head"])
+def test_gqa_group_reads_its_kv_head(attention):
     # G = 2: query heads 0,1 read kv head 0, heads 2,3 read kv head 1
     rng = np.random.default_rng(9)
     q = torch.tensor(rng.standard_normal((2, 4, 4)))
@@ -147,3 +153,14 @@ def test_linear_orientation():
     ref = [[sum(Wv[o][i] * x[r][i] for i in range(5)) for o in range(3)] for r in range(2)]
     for rowwise in (False, True):
         np.testing.assert_allclose(linear(torch.tensor(x), wb, rowwise).numpy(), ref, rtol=1e-12)
+
+
+def test_attention_forms_agree_on_long_ragged_rows():
+    rng = np.random.default_rng(21)
+    Q, H, Hkv, d, n = 9, 8, 2, 16, 700
+    q = torch.tensor(rng.standard_normal((Q, H, d)))
+    keys = torch.tensor(rng.standard_normal((Hkv, n + Q, d)))
+    vals = torch.tensor(rng.standard_normal((Hkv, n + Q, d)))
+    nv = [n + i + 1 for i in range(Q)]
+    np.testing.assert_allclose(attention_by_head(q, keys, vals, nv).numpy(), attention(q, keys, vals, nv).numpy(),
+                               rtol=1e-12, atol=1e-13)
