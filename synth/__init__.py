@@ -27,7 +27,7 @@ import numpy as np
 __all__ = [
     "ModelShape", "TINY", "TINY_QK", "QWEN3_8B", "tensor_specs", "make_weights",
     "make_prompt", "round_to_bf16_bits", "bf16_bits_to_f32", "planted_accepts",
-    "planted_drafts", "uniform_tokens", "normal_bf16",
+    "planted_accepts_stratified", "capped_geometric_mean", "planted_drafts", "uniform_tokens", "normal_bf16",
 ]
 
 
@@ -174,6 +174,31 @@ def planted_accepts(n_steps: int, mean: float, K: int, seed: int) -> np.ndarray:
     p = 1.0 / (mean + 1.0)
     a = g.geometric(p, size=n_steps) - 1  # numpy's geometric counts trials, support {1,2,...}
     return np.minimum(a, K).astype(np.int32)
+
+
+def capped_geometric_mean(mean: float, K: int) -> float:
+    """E[min(a, K)] for a ~ Geometric on {0,1,...} with E[a] = mean:
+    sum_{k=1..K} P(a >= k) = (1 - p) (1 - (1 - p)^K) / p with p = 1 / (mean + 1)."""
+    p = 1.0 / (mean + 1.0)
+    return (1.0 - p) * (1.0 - (1.0 - p) ** K) / p
+
+
+def planted_accepts_stratified(n_steps: int, mean: float, K: int, seed: int) -> np.ndarray:
+    """n_steps accept lengths of the same capped geometric law, drawn by stratified
+    sampling: the law's quantiles at u = (i + 1/2) / n_steps, i = 0..n_steps-1, in a
+    seeded random order. Their mean follows the law's mean to O(1/n_steps) rather than
+    O(1/sqrt(n_steps)), so a short timed window commits a reproducible number of tokens.
+
+    Quantile: the smallest k with P(a <= k) = 1 - (1 - p)^(k+1) >= u, i.e.
+    k = ceil(log(1 - u) / log(1 - p)) - 1, then capped at K.
+    """
+    p = 1.0 / (mean + 1.0)
+    u = (np.arange(n_steps, dtype=np.float64) + 0.5) / n_steps
+    k = np.ceil(np.log1p(-u) / np.log1p(-p)) - 1.0
+    a = np.clip(k, 0, K).astype(np.int32)
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=(0x57A,))))
+    g.shuffle(a)
+    return a
 
 
 def planted_drafts(stream: np.ndarray, n: int, a: int, K: int, vocab: int, rng: np.random.Generator) -> np.ndarray:

@@ -72,3 +72,22 @@ def test_planted_drafts_reproduce_the_planted_accept_length():
         if a < K:
             assert d[a] != stream[n + a + 1]
         assert accept_length(d.tolist(), greedy.tolist()) == a
+
+
+def test_stratified_accepts_follow_the_capped_geometric_law():
+    for mean, K in [(6.0, 32), (1.6, 8), (12.8, 64), (3.0, 4)]:
+        capped = synth.capped_geometric_mean(mean, K)
+        # the closed form against a direct sum of the capped law
+        p = 1.0 / (mean + 1.0)
+        pk = p * (1.0 - p) ** np.arange(K)
+        direct = float(np.sum(np.arange(K) * pk) + K * (1.0 - p) ** K)
+        assert abs(capped - direct) < 1e-9
+        a = synth.planted_accepts_stratified(4000, mean, K, seed=5)
+        assert a.min() == 0 and a.max() <= K
+        assert abs(a.mean() - capped) < 0.01 * max(1.0, capped)
+        assert abs(np.mean(a == 0) - p) < 1e-3  # the quantiles put a fraction p at zero
+        # a short window keeps its mean near the law's (stratified, not i.i.d.)
+        assert abs(synth.planted_accepts_stratified(147, mean, K, seed=6).mean() - capped) < 0.1 * max(1.0, capped)
+    a = synth.planted_accepts_stratified(64, 6.0, 32, seed=9)
+    assert np.array_equal(a, synth.planted_accepts_stratified(64, 6.0, 32, seed=9))
+    assert not np.array_equal(a, np.sort(a))  # seeded order, not sorted
