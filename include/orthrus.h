@@ -32,12 +32,17 @@
  *     (cache overrun, NaN logits, a bounded wait that ran out) are recorded in
  *     a sticky device int32 status word (first error wins), readable through
  *     orthrus_status_ptr(); kernels then stop writing the cache.
- *   - Matrices are row-major. bf16 = IEEE bfloat16 bits (uint16).
+ *   - Matrices are row-major. bf16 = IEEE bfloat16 bits (uint16); fp16 = IEEE
+ *     binary16 bits (uint16).
  *   - Model layout: W_qkv rows = q heads | k heads | v heads (each head_dim rows);
  *     W_gate_up rows = gate (d_ff) | up (d_ff); W_o [d_model][n_heads*head_dim];
  *     W_down [d_model][d_ff]; embed and lm_head [vocab][d_model] (untied).
- *   - KV cache: K and V bf16 [n_layers][batch][n_kv_heads][capacity][head_dim],
- *     post-QK-norm and post-RoPE; cache.len[b] (device int32) = live slots.
+ *   - KV cache: K and V [n_layers][batch][n_kv_heads][capacity][head_dim],
+ *     post-QK-norm and post-RoPE, rounded to bf16 values (the cache precision)
+ *     and held in the fp16 encoding, which represents every bf16 value of
+ *     magnitude in [2^-17, 65504] exactly (smaller ones to within 2^-25): one
+ *     tensor-core MMA takes operands of one type, and the attention's q and
+ *     softmax weights are fp16. cache.len[b] (device int32) = live slots.
  *   - Shapes supported by the kernels: head_dim in {64, 128}; d_model, d_ff and
  *     n_heads*head_dim multiples of 128; vocab a multiple of 128;
  *     n_heads / n_kv_heads in {1, 2, 4, 8}; 1 <= K <= 64.
@@ -99,8 +104,8 @@ typedef struct {
 
 /* The one shared KV cache (base view only). */
 typedef struct {
-  void* k;        /* bf16 [L][batch][Hkv][capacity][d] */
-  void* v;        /* bf16 [L][batch][Hkv][capacity][d] */
+  void* k;        /* fp16 encoding of bf16 values [L][batch][Hkv][capacity][d] */
+  void* v;        /* fp16 encoding of bf16 values [L][batch][Hkv][capacity][d] */
   int32_t* len;   /* device int32 [batch]: live slots per sequence */
   int32_t batch;
   int32_t capacity;
@@ -309,19 +314,59 @@ orthrus_status orthrus_decode_step_sampled(const void* plan, int32_t* pending, i
                                            float* draft_logits, float* verify_logits, int32_t* accept_len,
                                            int32_t* committed, orthrus_stream stream);
 
+/* ---- dynamic block size --------------------------------------------------
+ * The pages leave K to future work: choose it by how certain the generation
+ * is, larger for predictable text (code completion), smaller for open-ended
+ * text (news article, "Future Directions: Larger K and Higher Acceptance",
+ * item 1). Here certainty is the per-position acceptance rate alpha: a draft
+ * position is accepted with probability alpha until the first rejection, so a
+ * block of K drafts commits
+ *     E[a + 1 | K] = 1 + alpha + alpha^2 + ... + alpha^K
+ * tokens on average. Among candidate block sizes with measured step times, the
+ * policy picks the one that commits the most tokens per unit time, summed over
+ * the batch (one K serves every sequence of a launch). These calls run on the
+ * host only: no GPU, no stream; the caller feeds them the host copy of each
+ * step's accept lengths. */
+
+/* Running acceptance counts of one sequence, exponentially forgotten. */
+typedef struct {
+  float accepted; /* decayed sum of accepted drafts (the accept lengths a)        */
+  float rejected; /* decayed number of steps that ended in a rejection (a < K)    */
+} orthrus_accept_stats;
+
+/* stats[b] = decay * stats[b] + (a_b, 1 if a_b < K else 0) for b < batch, with a_b =
+ * accept_len[b] of a step run at block size K; a negative a_b (a failed step) leaves
+ * stats[b] unchanged. decay in (0, 1] (1 = plain counts). Errors: ORTHRUS_ERR_ARG
+ * (NULL pointers, batch < 1, K outside [0, 64], decay outside (0, 1], a_b > K). */
+orthrus_status orthrus_accept_stats_update(orthrus_accept_stats* stats, const int32_t* accept_len, int32_t batch,
+                                           int32_t K, float decay);
+
+/* alpha of one sequence: (accepted + 1) / (accepted + rejected + 2), the rate of the
+ * censored geometric counts under Laplace's rule of succession (1/2 with no data).
+ * Returns -1 for a NULL pointer or negative counts. */
+float orthrus_accept_rate(const orthrus_accept_stats* stats);
+
+/* The K among ks[0 .. n_options) that maximises sum_b E[a_b + 1 | K] / step_ms[i] with
+ * alpha_b = orthrus_accept_rate(&stats[b]); ties go to the smaller K. Every ks[i] in
+ * [1, 64] and step_ms[i] > 0 (the caller's measured time of one decode step at K = ks[i]).
+ * Returns that K, or -1 on bad arguments. */
+int32_t orthrus_choose_block_size(const orthrus_accept_stats* stats, int32_t batch, const int32_t* ks,
+                                  const float* step_ms, int32_t n_options);
+
 /* ---- single kernels, exposed for parity tests and microbenchmarks ------ */
 
 /* Block attention (the K1 kernel alone) for one layer's cache:
- *   q        bf16 [batch][Hkv][Q*G][d]: row i*G + g is query head kvh*G+g at block position i
+ *   q        fp16 [batch][Hkv][Q*G][d]: row i*G + g is query head kvh*G+g at block position i
  *            (post-norm, post-RoPE);
- *   k_cache, v_cache  bf16 [batch][Hkv][capacity][d];
- *   k_blk, v_blk      bf16 [batch][Hkv][blk_stride][d] (draft mode only: the
+ *   k_cache, v_cache  fp16 [batch][Hkv][capacity][d];
+ *   k_blk, v_blk      fp16 [batch][Hkv][blk_stride][d] (draft mode only: the
  *            block's own K/V, blk_stride >= Q);
  *   len      device int32 [batch]: cache rows [0, len[b]) precede the block;
  *   mode 0 = draft: every row sees cache[0,len) and block rows [0,Q);
  *   mode 1 = verify: the block's K/V already sit in cache slots [len, len+Q);
  *            row i sees cache[0, len+i].
- *   out      bf16 [batch][Q][H*d] (token-major, head h at columns h*d..).
+ *   out      bf16 [2][batch*Q][H*d] (token-major, head h at columns h*d..): the
+ *            result x as two planes, hi = bf16(x) then lo = bf16(x - hi).
  * Scratch comes from `workspace` (orthrus_attention_workspace_bytes). */
 size_t orthrus_attention_workspace_bytes(int32_t batch, int32_t n_kv_heads, int32_t group, int32_t Q, int32_t head_dim,
                                          int32_t capacity);

@@ -15,8 +15,10 @@
 //   warp 1: one thread issues S = Q K^T (tcgen05, K-major operands) into TMEM
 //           and then O_t = P V (V as an MN-major operand) into TMEM;
 //   warps 2-5: one thread per row: online softmax on S read from TMEM, P written
-//           as bf16 into shared memory in the 128-byte-swizzled K-major layout,
+//           as fp16 into shared memory in the 128-byte-swizzled K-major layout,
 //           O accumulated in registers with the running rescale.
+// Operands are fp16 (q, P, and K/V, whose bf16 values are held in the fp16
+// encoding); the output is written as two bf16 planes (hi, lo) for the O projection.
 // Chunks are combined by the last CTA to finish (atomic counter, fixed order).
 // Cache rows past the visible range inside a loaded tile (stale, NaN-poisoned or
 // never written) are masked out of S and their V rows zeroed before P V, so they
@@ -39,7 +41,8 @@ struct AttnArgs {
   int max_chunks;              // gridDim.x
   float scale_log2;            // log2(e) / sqrt(d)
   const int* len;
-  __nv_bfloat16* out;          // [nb][Q][H*d]
+  __nv_bfloat16* out;          // [2][nb*Q][H*d]: hi plane, then the lo plane at + out_lo
+  size_t out_lo;
   float* part_o;               // [nb*Hkv*row_tiles][max_chunks][128][d]
   float2* part_ml;             // [nb*Hkv*row_tiles][max_chunks][128]
   int* counter;                // [nb*Hkv*row_tiles], zero between launches
@@ -59,11 +62,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   constexpr int d = D;
-  const uint32_t tile_bytes = 128u * d * 2u;  // 128 rows x d bf16
+  const uint32_t tile_bytes = 128u * d * 2u;  // 128 rows x d fp16
   uint8_t* sQ = smem;
   uint8_t* sK[2] = {smem + tile_bytes, smem + 3 * tile_bytes};
   uint8_t* sV[2] = {smem + 2 * tile_bytes, smem + 4 * tile_bytes};
-  uint8_t* sP = smem + 5 * tile_bytes;  // 128 rows x 128 keys bf16 = 32 KB
+  uint8_t* sP = smem + 5 * tile_bytes;  // 128 rows x 128 keys fp16 = 32 KB
   uint64_t* bars = (uint64_t*)(sP + 128 * 128 * 2);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [2]
@@ -168,8 +171,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idS = idesc_bf16(128, 128, false);
-      const uint32_t idO = idesc_bf16(128, d, true);
+      const uint32_t idS = idesc_f16(128, 128, false);  // fp16 q and K
+      const uint32_t idO = idesc_f16(128, d, true);      // fp16 P and V
       bool ok = mbar_wait(q_full, 0, a.status);
       const uint32_t qa = smem_u32(sQ), pa = smem_u32(sP);
       for (int j = 0; ok && j < n_tiles; ++j) {
@@ -180,14 +183,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t ka = smem_u32(sK[s]), va = smem_u32(sV[s]);
         for (int kk = 0; kk < d / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tS, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          mma_ss(tS, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
         if (!mbar_wait(p_full, j & 1, a.status)) break;
         tc_fence_after();
         for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
           const uint32_t poff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tO, sw128_desc(pa + poff, 16, 1024), sw128_desc(va + kk * 2048, 16384, 1024), idO,
+          mma_ss(tO, sw128_desc(pa + poff, 16, 1024), sw128_desc(va + kk * 2048, 16384, 1024), idO,
                       kk > 0 ? 1u : 0u);
         }
         mma_commit(o_full);
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const float m_new = fmaxf(m_run, mx);
       const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
-      // pass 2: P = exp2(s - m_new) as bf16 into the swizzled P tile
+      // pass 2: P = exp2(s - m_new) as fp16 into the swizzled P tile
       float sum = 0.f;
       for (int c0 = 0; c0 < 128; c0 += 32) {
         float v[32];
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float p0 = (key0 + c0 + t < lim) ? exp2f(v[t] * a.scale_log2 - m_new) : 0.f;
           const float p1 = (key0 + c0 + t + 1 < lim) ? exp2f(v[t + 1] * a.scale_log2 - m_new) : 0.f;
           sum += p0 + p1;
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          __half2 h2 = __floats2half2_rn(p0, p1);
           pk[t / 2] = *reinterpret_cast<uint32_t*>(&h2);
         }
         // keys c0..c0+31 = four 16-byte chunks of row r in atom column c0/64
@@ -303,10 +306,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
           for (int e = 0; e < d; e += 8) {
-            __nv_bfloat162 h[4];
+            float y8[8];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(o[e + 2 * t] * inv, o[e + 2 * t + 1] * inv);
-            *reinterpret_cast<uint4*>(dst + e) = *reinterpret_cast<uint4*>(h);
+            for (int t = 0; t < 8; ++t) y8[t] = o[e + t] * inv;
+            st_split_x8(dst + e, dst + a.out_lo + e, y8);
           }
         }
       } else {
@@ -349,10 +352,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
             for (int e = 0; e < d; e += 8) {
-              __nv_bfloat162 h[4];
+              float y8[8];
 #pragma unroll
-              for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(o[e + 2 * t] * inv, o[e + 2 * t + 1] * inv);
-              *reinterpret_cast<uint4*>(dst + e) = *reinterpret_cast<uint4*>(h);
+              for (int t = 0; t < 8; ++t) y8[t] = o[e + t] * inv;
+              st_split_x8(dst + e, dst + a.out_lo + e, y8);
             }
           }
         }

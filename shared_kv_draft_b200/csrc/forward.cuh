@@ -14,28 +14,38 @@
 // weight stream does not stop at phase boundaries.
 //
 // Phases of one forward (phase p depends on the previous active phase only):
-//   EMBED         h = E[ids], xg = bf16(h * gamma_attn[0]), per-row sums of squares
+//   EMBED         h = E[ids], xg = split(h * gamma_attn[0]), per-row sums of squares
 //   per layer:
 //     QKV         [xg] W_qkv^T, * rstd, per-head q/k RMSNorm, RoPE; q -> qbuf, K/V ->
 //                 cache slots len+i (verify) or the draft block scratch (draft)
 //     ATTN        block attention over (sequence, kv head, 128-row tile, key chunk) units
 //     COMBINE     merge of the key-chunk partials (only when some slot has several chunks)
-//     O           h += attn W_o^T; xg = bf16(h * gamma_mlp); sums of squares
+//     O           h += attn W_o^T; xg = split(h * gamma_mlp); sums of squares
 //     GU          act = silu(rstd * xg W_g^T) * (rstd * xg W_u^T)
-//     DOWN        h += act W_down^T; xg = bf16(h * gamma_next); sums of squares
+//     DOWN        h += act W_down^T; xg = split(h * gamma_next); sums of squares
 //   LM            logits = rstd * xg W_lm^T; running argmax per row
 // RMSNorm is folded into its neighbours: RMSNorm(h) W^T = diag(rstd) (h*gamma) W^T,
-// so the residual epilogue writes bf16(h * gamma) and 128-column partial sums of
+// so the residual epilogue writes split(h * gamma) and 128-column partial sums of
 // h^2, and the consumer multiplies its accumulator rows by rstd, computed from the
 // partial sums in a fixed order (deterministic).
+//
+// Operand precision. Over 36 layers every bf16 rounding of an activation adds to the
+// logits' error, so the operands carry more bits than bf16:
+//   - an activation that feeds a layer projection (xg, the attention output, the SwiGLU
+//     output) is written as two bf16 planes, hi = bf16(x) and lo = bf16(x - hi); every
+//     weight chunk is multiplied with both (two MMAs into one fp32 accumulator), so the
+//     projection sees x to about 2^-17 relative. The LM head reads the hi plane only;
+//   - attention runs on fp16 operands: q and the softmax weights P (11 significant bits),
+//     and K/V, bf16 values held in the fp16 encoding.
 //
 // Warp roles (224 threads): warp 0 = TMA producer of weight tiles, warp 6 = TMA
 // producer of activation tiles (the loads that wait for the previous phase), warp
 // 1 = tcgen05.mma issuer, warps 2-5 = epilogue (TMEM -> registers -> fused
 // epilogue), attention softmax, embedding and chunk merge. Two issuing threads
 // matter: one thread issuing 8 KB copies streams about 4 TB/s, two reach the
-// HBM rate. Ring stage = a 16 KB "A" slot (a weight tile of 128
-// rows x 64 k, or an attention Q / K / V tile) + an activation slot of Mt x 64.
+// HBM rate. Ring stage = a 32 KB slot (a weight box of 128 rows x two 64-wide k
+// chunks, or an attention K / V tile) + an activation slot of Mt rows x two k chunks x
+// two planes.
 #pragma once
 #include "gemm.cuh"
 
@@ -75,14 +85,16 @@ enum {
   G_VC64,
   G_KB64,
   G_VB64,
-  G_XN,
-  G_ATTN = G_XN + 8,
-  G_ACT = G_ATTN + 8,
-  G_LM3 = G_ACT + 8,  // 3-D views of the LM head and of the activations (k-pair boxes)
-  G_XN3,
-  G_ATTN3 = G_XN3 + 8,
-  G_ACT3 = G_ATTN3 + 8,
-  G_COUNT = G_ACT3 + 8
+  G_XN,                 // normalised input, hi plane only (the LM head's operand)
+  G_XNP = G_XN + 8,     // normalised input, both planes: (64 columns, rows, plane)
+  G_ATTN = G_XNP + 8,   // attention output, both planes
+  G_ACT = G_ATTN + 8,   // SwiGLU output, both planes
+  G_LM3 = G_ACT + 8,    // k-pair views of the LM head and of the activations (persistent kernel)
+  G_XN3,                // hi plane: (64 columns, rows, k chunk)
+  G_XN4 = G_XN3 + 8,    // both planes: (64 columns, rows, k chunk, plane)
+  G_ATTN4 = G_XN4 + 8,
+  G_ACT4 = G_ATTN4 + 8,
+  G_COUNT = G_ACT4 + 8
 };
 
 enum PhaseKind : int { PH_EMBED = 0, PH_QKV, PH_ATTN, PH_COMBINE, PH_O, PH_GU, PH_DOWN, PH_LM };
@@ -117,12 +129,13 @@ struct FwdArgs {
   int* len;                  // [batch] (read; the fused accept advances it)
   const __nv_bfloat16* embed;
   const float* final_norm;
-  __nv_bfloat16 *kc, *vc, *blk_k, *blk_v;
+  __half *kc, *vc, *blk_k, *blk_v;  // bf16 values in the fp16 encoding
   float* h;                  // [rows][D]
-  __nv_bfloat16* xg;         // [rows][D]
-  __nv_bfloat16* qbuf;       // [nb][Hkv][Q*G][d]
-  __nv_bfloat16* attn;       // [rows][H*d]
-  __nv_bfloat16* act;        // [rows][F]
+  __nv_bfloat16* xg;         // [2][rows][D]: hi plane, then lo plane at + xg_lo
+  __half* qbuf;              // [nb][Hkv][Q*G][d]
+  __nv_bfloat16* attn;       // [2][rows][H*d] (lo plane at + attn_lo)
+  __nv_bfloat16* act;        // [2][rows][F] (lo plane at + act_lo)
+  size_t xg_lo, attn_lo, act_lo;  // element offsets of the lo planes
   float2* rope;              // [rows][d/2]
   float* ss;                 // [D/128][ss_ld] partial sums of squares
   int ss_ld;
@@ -198,8 +211,9 @@ __host__ inline size_t fwd_fixed_smem(int d) {
          128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/ +
          kMaxGrid * 4 /*unit-range starts*/;
 }
-// ring stage: 32 KB weight box (128 rows x two k chunks) + activation box (Mt rows x two k chunks)
-__host__ inline size_t fwd_stage_bytes(int Mt) { return 32768 + (size_t)Mt * 256; }
+// ring stage: 32 KB weight box (128 rows x two k chunks) + activation box (Mt rows x two k
+// chunks x two planes; the LM head reads the hi plane only)
+__host__ inline size_t fwd_stage_bytes(int Mt) { return 32768 + (size_t)Mt * 512; }
 
 // Shared state every role derives identically at kernel start.
 struct FwdGeom {
@@ -219,6 +233,7 @@ struct GemmPhase {
   const CUtensorMap* mw;
   const CUtensorMap* mx;
   int gu;             // SwiGLU tile layout (64 gate + 64 up rows)
+  int planes;         // activation planes: 2 (hi + lo) for the layer projections, 1 for the LM head
 };
 
 __device__ inline GemmPhase gemm_phase(const FwdArgs& a, int kind, int l) {
@@ -227,37 +242,39 @@ __device__ inline GemmPhase gemm_phase(const FwdArgs& a, int kind, int l) {
   const CUtensorMap* gm = a.maps + (size_t)a.L * M_PER_LAYER;
   const bool draft = a.view == VIEW_DRAFT;
   g.gu = 0;
+  g.planes = 2;
   if (kind == PH_QKV) {
     g.epi = EPI_QKV;
     g.n_tiles = (a.H + 2 * a.Hkv) * a.d / 128;
     g.k_chunks = a.D / 128;
     g.mw = lm + (draft ? M_WDQKV3 : M_WQKV3);
-    g.mx = gm + G_XN3 + a.mt_idx;
+    g.mx = gm + G_XN4 + a.mt_idx;
   } else if (kind == PH_O) {
     g.epi = EPI_RESID;
     g.n_tiles = a.D / 128;
     g.k_chunks = a.H * a.d / 128;
     g.mw = lm + (draft ? M_WDO3 : M_WO3);
-    g.mx = gm + G_ATTN3 + a.mt_idx;
+    g.mx = gm + G_ATTN4 + a.mt_idx;
   } else if (kind == PH_GU) {
     g.epi = EPI_SWIGLU;
     g.n_tiles = a.F / 64;
     g.k_chunks = a.D / 128;
     g.mw = lm + M_WGU4;
-    g.mx = gm + G_XN3 + a.mt_idx;
+    g.mx = gm + G_XN4 + a.mt_idx;
     g.gu = 1;
   } else if (kind == PH_DOWN) {
     g.epi = EPI_RESID;
     g.n_tiles = a.D / 128;
     g.k_chunks = a.F / 128;
     g.mw = lm + M_WDOWN3;
-    g.mx = gm + G_ACT3 + a.mt_idx;
+    g.mx = gm + G_ACT4 + a.mt_idx;
   } else {  // PH_LM
     g.epi = EPI_ARGMAX;
     g.n_tiles = a.V / 128;
     g.k_chunks = a.D / 128;
     g.mw = gm + G_LM3;
     g.mx = gm + G_XN3 + a.mt_idx;
+    g.planes = 1;
   }
   g.units = (long long)g.n_tiles * g.k_chunks;
   return g;
@@ -349,19 +366,6 @@ __device__ inline AttUnit att_unit(const FwdArgs& a, const FwdGeom& g, const int
 // the q/k/v epilogue (so a head's sum of squares is two shuffles). Every thread
 // then runs the same short code and stores 16-byte vectors.
 
-// 16 floats -> 8 packed bf16 pairs -> two 16-byte stores
-__device__ __forceinline__ void st_bf16x16(__nv_bfloat16* dst, const float* x) {
-  uint32_t w[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h2);
-  }
-  uint4* p = reinterpret_cast<uint4*>(dst);
-  p[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  p[1] = make_uint4(w[4], w[5], w[6], w[7]);
-}
-
 // Scratch layout of the epilogues (floats): the 32-row staging tile [32][kEpiStride],
 // 128 per-quarter sums, then the second group's staging [4][kEpiStride] and its 16
 // per-quarter sums. The second group carries token rows [m0+32, m0+32+n2), n2 <= 4:
@@ -412,8 +416,8 @@ __device__ __forceinline__ float resid_quarter(const FwdArgs& a, const float* sr
       y[4 * c] *= g4.x, y[4 * c + 1] *= g4.y, y[4 * c + 2] *= g4.z, y[4 * c + 3] *= g4.w;
     }
     __nv_bfloat16* xp = a.xg + (size_t)m * D + nt * 128 + qq * 32;
-    st_bf16x16(xp, y);
-    st_bf16x16(xp + 16, y + 16);
+    st_split_x16(xp, xp + a.xg_lo, y);
+    st_split_x16(xp + 16, xp + a.xg_lo + 16, y + 16);
   }
   return (s0 + s1) + (s2 + s3);
 }
@@ -471,7 +475,7 @@ __device__ __forceinline__ void fwd_resid_epilogue(const FwdArgs& a, const float
 // factors of token rows [0, rope_rows) (both in shared memory; rows past
 // rope_rows read the global table).
 struct QkvCtx {
-  __nv_bfloat16 *kdst, *vdst;
+  __half *kdst, *vdst;
   int kv_stride;
   const float* gains;
   const float2* rope;
@@ -550,7 +554,7 @@ __device__ __forceinline__ void qkv_item(const FwdArgs& a, const QkvCtx& q, cons
   }
   if (valid) {
     const int bb = a.nb == 1 ? 0 : m / a.Q, i = m - bb * a.Q;  // (runtime divides cost ~100 cycles each)
-    __nv_bfloat16* dst = nullptr;
+    __half* dst = nullptr;
     if (kind == 0) {
       const int G = a.G;
       const int kvh = (G & (G - 1)) == 0 ? hh >> (31 - __clz(G)) : hh / G, g = hh - kvh * G;
@@ -560,10 +564,15 @@ __device__ __forceinline__ void qkv_item(const FwdArgs& a, const QkvCtx& q, cons
       const int slot = a.view == VIEW_DRAFT ? i : lens_s[bb] + i;
       if (slot >= 0 && slot < q.kv_stride)
         dst = (kind == 1 ? q.kdst : q.vdst) + ((size_t)(bb * a.Hkv + kvh) * q.kv_stride + slot) * d;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {  // K and V keep bf16 values (the cache precision)
+        x1[e] = kv_value(x1[e]);
+        x2[e] = kv_value(x2[e]);
+      }
     }
     if (dst) {
-      st_bf16x16(dst + e0, x1);
-      st_bf16x16(dst + half + e0, x2);
+      st_f16x16(dst + e0, x1);
+      st_f16x16(dst + half + e0, x2);
     }
   }
 }
@@ -608,7 +617,8 @@ __device__ __forceinline__ void swiglu_item(const FwdArgs& a, const float* src, 
     for (int i = 0; i < 4; ++i)  // fast reciprocal: an IEEE divide branches per element
       y[4 * c + i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * u[i];
   }
-  st_bf16x16(a.act + (size_t)m * a.F + nt * 64 + 16 * qq, y);
+  __nv_bfloat16* dst = a.act + (size_t)m * a.F + nt * 64 + 16 * qq;
+  st_split_x16(dst, dst + a.act_lo, y);
 }
 
 __device__ __forceinline__ void fwd_swiglu_epilogue(const FwdArgs& a, const float* v, const float* v2, int row, int m0,
@@ -867,7 +877,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           const int col = pp * 128 + et;
           const float x = __bfloat162float(src[col]);
           a.h[(size_t)m * D + col] = x;
-          a.xg[(size_t)m * D + col] = __float2bfloat16(x * g0[col]);
+          const float xv = x * g0[col];
+          const __nv_bfloat16 xh = __float2bfloat16(xv);
+          a.xg[(size_t)m * D + col] = xh;
+          a.xg[a.xg_lo + (size_t)m * D + col] = __float2bfloat16(xv - __bfloat162float(xh));
           const float s = warp_sum(x * x);
           if (lane == 0) epi[ew * 64 + pp] = s;
         }
@@ -1151,6 +1164,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         int cc0 = c_lo + 1, s0, s1;
         gather2(cc0, c_hi, s0, s1, t);
+        const int f0 = s0, f1 = s1;  // the first round's slots (s0, s1 move on in later rounds)
         float4 x[2][8];
         load2(x, s0, s1, 0);
         // a second token group (the 33rd row of a K = 32 verify block) is usually one float4
@@ -1193,7 +1207,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             // the first round's contributors: row 8 prefetched, rows 9.. (tokens 36..) loaded here
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-              const int sl = q == 0 ? s0 : s1;
+              const int sl = q == 0 ? f0 : f1;
               const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
                                  8 * 128 + row;
               v[0] += x2[q].x;
@@ -1330,7 +1344,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               const float p1 = fast_exp2(c0 + tt + 1 < nv ? sv[tt + 1] * a.scale_log2 - m_new : -INFINITY);
               sum0 += p0;
               sum1 += p1;
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              __half2 h2 = __floats2half2_rn(p0, p1);
               pk[tt / 2] = *reinterpret_cast<uint32_t*>(&h2);
             }
             uint8_t* rowp = scr + row * 128;
@@ -1382,10 +1396,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             const float inv = l_run > 0.f ? __fdividef(1.f, l_run) : 0.f;
 #pragma unroll
             for (int e = 0; e < d; e += 8) {
-              __nv_bfloat162 hb[4];
+              float y8[8];
 #pragma unroll
-              for (int tt = 0; tt < 4; ++tt) hb[tt] = __floats2bfloat162_rn(o[e + 2 * tt] * inv, o[e + 2 * tt + 1] * inv);
-              *reinterpret_cast<uint4*>(dst + e) = *reinterpret_cast<uint4*>(hb);
+              for (int tt = 0; tt < 8; ++tt) y8[tt] = o[e + tt] * inv;
+              st_split_x8(dst + e, dst + a.attn_lo + e, y8);
             }
           }
         } else {
@@ -1462,10 +1476,10 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           __nv_bfloat16* dst = a.attn + ((size_t)(bb * a.Q + i) * a.H + kvh * a.G + gg) * d + sub * per;
 #pragma unroll
           for (int e = 0; e < per; e += 8) {
-            __nv_bfloat162 hb[4];
+            float y8[8];
 #pragma unroll
-            for (int tt = 0; tt < 4; ++tt) hb[tt] = __floats2bfloat162_rn(acc[e + 2 * tt] * inv, acc[e + 2 * tt + 1] * inv);
-            *reinterpret_cast<uint4*>(dst + e) = *reinterpret_cast<uint4*>(hb);
+            for (int tt = 0; tt < 8; ++tt) y8[tt] = acc[e + tt] * inv;
+            st_split_x8(dst + e, dst + a.attn_lo + e, y8);
           }
         }
         signal(p);
@@ -1486,7 +1500,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   constexpr int d = D_HEAD;
   constexpr int halves = d / 64;
   const int S = a.stages;
-  const uint32_t x_bytes = (uint32_t)a.Mt * 256u;  // two k chunks of Mt rows
+  const uint32_t x_bytes = (uint32_t)a.Mt * 512u;  // two k chunks x two planes of Mt rows
   const uint32_t stage_bytes = 32768u + x_bytes;
   uint8_t* sQ = smem + (size_t)S * stage_bytes;   // attention Q tile, d/64 blocks of 128 rows x 64
   uint8_t* scr = sQ + (size_t)128 * d * 2;         // P tile / epilogue staging
@@ -1629,8 +1643,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 break;
               }
               if (u == u0) tl_mark<TL>(a, n_ph, p, TL_X0);
-              mbar_arrive_expect_tx(&full[s], x_bytes);
-              tma_load_3d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k);
+              // box [plane][k chunk][Mt rows][64]
+              mbar_arrive_expect_tx(&full[s], (uint32_t)a.Mt * 256u * (uint32_t)gp.planes);
+              if (gp.planes == 2) tma_load_4d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k, 0);
+              else tma_load_3d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k);
             }
             last_ph[s] = (int)ph;
           }
@@ -1713,8 +1729,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
     // ======================= MMA issuer =======================
     if (lane == 0) {
       const uint32_t idesc_g = idesc_bf16(128, a.Mt, false);
-      const uint32_t idS = idesc_bf16(128, 64, false);
-      const uint32_t idO = idesc_bf16(128, d, true);
+      const uint32_t idS = idesc_f16(128, 64, false);  // fp16 q and K
+      const uint32_t idO = idesc_f16(128, d, true);    // fp16 P and V
       const uint32_t pa = smem_u32(scr);
       int it = 0, seg = 0, ta = 0, qu = 0;
       bool ok = true;
@@ -1753,13 +1769,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               tc_fence_after();
               const uint32_t wa = smem_u32(stage_ptr(s));
               const uint32_t xa = wa + 32768;
+              const uint32_t x_lo = 2u * (uint32_t)a.Mt * 128u;  // lo plane after the hi plane's two chunks
 #pragma unroll
               for (int c2 = 0; c2 < 2; ++c2) {  // the two 64-wide k chunks of the unit
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_bf16_ss(d_tmem, sw128_desc(wa + c2 * 16384 + kk * 32, 16, 1024),
-                              sw128_desc(xa + c2 * (uint32_t)a.Mt * 128u + kk * 32, 16, 1024), idesc_g,
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t wd = sw128_desc(wa + c2 * 16384 + kk * 32, 16, 1024);
+                  const uint32_t xo = c2 * (uint32_t)a.Mt * 128u + kk * 32;
+                  mma_ss(d_tmem, wd, sw128_desc(xa + xo, 16, 1024), idesc_g,
                               (u > seg_start || c2 > 0 || kk > 0) ? 1u : 0u);
+                  if (gp.planes == 2) mma_ss(d_tmem, wd, sw128_desc(xa + x_lo + xo, 16, 1024), idesc_g, 1u);
+                }
               }
               mma_commit(&empty[s]);
             }
@@ -1790,7 +1810,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               const uint32_t ka = smem_u32(stage_ptr(ks));
 #pragma unroll
               for (int kk = 0; kk < d / 16; ++kk)
-                mma_bf16_ss(tS, sw128_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                mma_ss(tS, sw128_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                             sw128_desc(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
               mma_commit(s_full);
               mma_commit(&empty[ks]);
@@ -1811,7 +1831,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               const uint32_t va = smem_u32(stage_ptr(vs));
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, 8192, 1024), idO,
+                mma_ss(tO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, 8192, 1024), idO,
                             (j > 0 || kk > 0) ? 1u : 0u);
               mma_commit(o_full);
               mma_commit(&empty[vs]);

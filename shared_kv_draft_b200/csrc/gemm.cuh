@@ -18,9 +18,12 @@
 //    arrives last (atomic counter, no waiting): it sums all fp32 partials in a
 //    fixed k order, so results do not depend on arrival order.
 //  * Epilogues: fp32 store, residual add into the fp32 hidden state, per-head
-//    q/k RMSNorm + RoPE + bf16 store of q and of K/V into the cache (or the
-//    draft block scratch), SwiGLU (each tile holds 64 gate rows and the 64
-//    matching up rows), and LM-head argmax (64-bit max of (value, -index)).
+//    q/k RMSNorm + RoPE + fp16 store of q and of K/V (bf16 values) into the
+//    cache (or the draft block scratch), SwiGLU (each tile holds 64 gate rows
+//    and the 64 matching up rows; hi and lo planes out), and LM-head argmax
+//    (64-bit max of (value, -index)).
+//  * X may come in two bf16 planes (hi + lo of one fp32 activation): each
+//    weight chunk is multiplied with both into the same fp32 accumulator.
 #pragma once
 #include "ptx.cuh"
 
@@ -40,9 +43,9 @@ struct QkvEpi {
   const float* gk;           // [d]
   const float2* rope;        // [M][d/2] (cos, sin) of each token row's position
   const int* len;            // [batch] cache lengths
-  __nv_bfloat16* qbuf;       // [nb][Hkv][Q*G][d]
-  __nv_bfloat16* kdst;       // this layer's K destination [batch][Hkv][kv_stride][d]
-  __nv_bfloat16* vdst;
+  __half* qbuf;              // [nb][Hkv][Q*G][d], fp16
+  __half* kdst;              // this layer's K destination [batch][Hkv][kv_stride][d] (bf16 values, fp16 encoding)
+  __half* vdst;
   int kv_stride;             // capacity (cache) or block-scratch rows
 };
 
@@ -52,13 +55,15 @@ struct GemmArgs {
   int m_tiles, n_tiles, k_chunks;
   long long total_units;
   int stages;
+  int planes;                // activation planes of X: 2 (hi + lo, two MMAs per chunk) or 1
   int swiglu_F;              // SwiGLU: row offset of the up rows in W
   float* partial;            // [2 * grid][128 rows][Mt] fp32 partial sums of split tiles
   int* tile_counter;         // [m_tiles * n_tiles], zero between launches
   int* status;
   float* out_f32;            // STORE: Y[M][ld_out]; RESID: h[M][ld_out] (+=)
   int ld_out;
-  __nv_bfloat16* out_bf16;   // SWIGLU: act[M][ld_out]
+  __nv_bfloat16* out_bf16;   // SWIGLU: act[2][M][ld_out], hi plane then the lo plane at + out_lo
+  size_t out_lo;
   QkvEpi qkv;
   unsigned long long* amax;  // ARGMAX: [M] running keys
   float* logits;             // ARGMAX: optional fp32 [M][ld_logits]
@@ -75,8 +80,9 @@ __device__ inline int unit_owner(long long u, long long W, int G) {
   return c;
 }
 
-__host__ inline size_t gemm_smem_bytes(int Mt, int stages) {
-  return 1024 /*align*/ + (size_t)stages * (16384 + Mt * 128) + 32 * kEpiStride * 4 + 4 * 32 * 8 + 2 * 16 * 8 + 128;
+__host__ inline size_t gemm_smem_bytes(int Mt, int stages, int planes) {
+  return 1024 /*align*/ + (size_t)stages * (16384 + (size_t)Mt * 128 * planes) + 32 * kEpiStride * 4 + 4 * 32 * 8 +
+         2 * 16 * 8 + 128;
 }
 
 // --------------------------------------------------------------------------
@@ -113,7 +119,11 @@ __device__ __forceinline__ void epilogue_group(const GemmArgs& a, float* v, int 
           const float g = v[j];
           const float u = epi[j * kEpiStride + row];
           const float s = g / (1.0f + __expf(-g));
-          a.out_bf16[(size_t)(mt * 128 + m) * a.ld_out + nt * 64 + row] = __float2bfloat16(s * u);
+          const float y = s * u;
+          const __nv_bfloat16 yh = __float2bfloat16(y);
+          const size_t o = (size_t)(mt * 128 + m) * a.ld_out + nt * 64 + row;
+          a.out_bf16[o] = yh;
+          a.out_bf16[a.out_lo + o] = __float2bfloat16(y - __bfloat162float(yh));
         }
       }
     }
@@ -167,19 +177,19 @@ __device__ __forceinline__ void epilogue_group(const GemmArgs& a, float* v, int 
         }
         if (kind == 0) {
           const int kvh = hh / G, g = hh - kvh * G;
-          __nv_bfloat16* dst = q.qbuf + ((size_t)(bb * q.Hkv + kvh) * (q.Q * G) + i * G + g) * d;
+          __half* dst = q.qbuf + ((size_t)(bb * q.Hkv + kvh) * (q.Q * G) + i * G + g) * d;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            if (k < nper) dst[lane + 32 * k] = __float2bfloat16(x[k]);
+            if (k < nper) dst[lane + 32 * k] = __float2half_rn(x[k]);
         } else {
           const int kvh = hh - q.H - (kind == 2 ? q.Hkv : 0);
           const int slot = q.mode == VIEW_DRAFT ? i : q.len[b] + i;
           if (slot >= 0 && slot < q.kv_stride) {
-            __nv_bfloat16* base = kind == 1 ? q.kdst : q.vdst;
-            __nv_bfloat16* dst = base + ((size_t)(b * q.Hkv + kvh) * q.kv_stride + slot) * d;
+            __half* base = kind == 1 ? q.kdst : q.vdst;
+            __half* dst = base + ((size_t)(b * q.Hkv + kvh) * q.kv_stride + slot) * d;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              if (k < nper) dst[lane + 32 * k] = __float2bfloat16(x[k]);
+              if (k < nper) dst[lane + 32 * k] = __float2half_rn(kv_value(x[k]));
           }
         }
       }
@@ -216,7 +226,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int S = a.stages;
-  const uint32_t x_bytes = (uint32_t)a.Mt * 128u;
+  const uint32_t x_bytes = (uint32_t)a.Mt * 128u * (uint32_t)a.planes;  // [plane][Mt rows][64]
   const uint32_t stage_bytes = 16384u + x_bytes;
   float* epi = (float*)(smem + (size_t)S * stage_bytes);
   unsigned long long* red = (unsigned long long*)(epi + 32 * kEpiStride);
@@ -282,7 +292,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int t = (int)(u / kc), k = (int)(u - (long long)t * kc);
         const int mt = t - (t / a.m_tiles) * a.m_tiles;
         uint8_t* xdst = smem + (size_t)s * stage_bytes + 16384;
-        tma_load_2d_hint(xdst, &tmX, &full[s], k * 64, mt * 128, pol_x);  // one box of Mt token rows
+        if (a.planes == 2) tma_load_3d(xdst, &tmX, &full[s], k * 64, mt * 128, 0);  // Mt rows of both planes
+        else tma_load_2d_hint(xdst, &tmX, &full[s], k * 64, mt * 128, pol_x);  // one box of Mt token rows
       };
       // weights never depend on earlier kernels: fill the ring with weight tiles
       // before waiting for the predecessor, then add the activation tiles
@@ -332,10 +343,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t wa = smem_u32(smem + (size_t)s * stage_bytes);
           const uint32_t xa = wa + 16384;
+          const uint32_t x_lo = (uint32_t)a.Mt * 128u;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(d_tmem, sw128_desc(wa + kk * 32, 16, 1024), sw128_desc(xa + kk * 32, 16, 1024), idesc,
-                        (u > seg_start || kk > 0) ? 1u : 0u);
+            const uint64_t wd = sw128_desc(wa + kk * 32, 16, 1024);
+            mma_ss(d_tmem, wd, sw128_desc(xa + kk * 32, 16, 1024), idesc, (u > seg_start || kk > 0) ? 1u : 0u);
+            if (a.planes == 2) mma_ss(d_tmem, wd, sw128_desc(xa + x_lo + kk * 32, 16, 1024), idesc, 1u);
           }
           mma_commit(&empty[s]);
         }

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "attention.cuh"
 #include "forward.cuh"
@@ -17,6 +18,7 @@
 #include "orthrus.h"
 #include "sampling.cuh"
 #include "small.cuh"
+#include "policy.cuh"
 
 using namespace orthrus;
 
@@ -41,29 +43,34 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D bf16 map over a row-major [rows][cols] matrix; box = box_cols x box_rows, 128-byte swizzle.
-bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+constexpr CUtensorMapDataType kF16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+
+// 2D map of 16-bit elements over a row-major [rows][cols] matrix; box = box_cols x box_rows,
+// 128-byte swizzle.
+bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+           CUtensorMapDataType dt = kBF16) {
   EncodeTiledFn f = encode_fn();
   if (!f || !base) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  return f(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D bf16 map over [z][rows][cols]; box = 64 cols x box_rows rows x box_z.
+// 3D map of 16-bit elements over [z][rows][cols]; box = 64 cols x box_rows rows x box_z.
 bool map3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t z, uint32_t box_rows = 128,
-           uint32_t box_z = 1) {
+           uint32_t box_z = 1, CUtensorMapDataType dt = kBF16) {
   EncodeTiledFn f = encode_fn();
   if (!f || !base) return false;
   cuuint64_t dims[3] = {cols, rows, z};
   cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
   cuuint32_t box[3] = {64, box_rows, box_z};
   cuuint32_t es[3] = {1, 1, 1};
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  return f(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -94,6 +101,24 @@ bool map_kpair(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
   return map_nd(m, base, 3, dims, strides, box);
 }
 
+// An activation in two planes [2][rows][cols] (hi, then lo), as (64 columns, rows, plane): a box
+// of (64, box_rows, 2) is one 64-wide k chunk of both planes.
+bool map_planes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[3] = {cols, rows, 2};
+  const uint64_t strides[2] = {cols * 2, cols * rows * 2};
+  const uint32_t box[3] = {64, box_rows, 2};
+  return map_nd(m, base, 3, dims, strides, box);
+}
+
+// The same as (64 columns, rows, cols/64 chunks, plane): a box of (64, box_rows, 2, 2) is two
+// consecutive 64-wide k chunks of both planes, laid out [plane][chunk][row][64].
+bool map_kpair_planes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  const uint64_t dims[4] = {64, rows, cols / 64, 2};
+  const uint64_t strides[3] = {cols * 2, 128, cols * rows * 2};
+  const uint32_t box[4] = {64, box_rows, 2, 2};
+  return map_nd(m, base, 4, dims, strides, box);
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int round_up(int x, int a) { return (x + a - 1) / a * a; }
 int next_pow2(int x) {
@@ -114,17 +139,8 @@ int num_sms() {
 
 constexpr size_t kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100
 
-// Programmatic dependent launch for every kernel (ORTHRUS_PDL=0 in the
-// environment turns it off): a kernel may begin its prologue and weight loads
-// while its predecessor drains; its griddepcontrol.wait orders everything else.
-bool pdl_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("ORTHRUS_PDL");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
-}
+// Programmatic dependent launch for every kernel: a kernel may begin its prologue and
+// weight loads while its predecessor drains; its griddepcontrol.wait orders everything else.
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
@@ -138,7 +154,7 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -160,13 +176,15 @@ struct alignas(64) Plan {
   const void* embed;
   const float* final_norm;
   const void* lm_head;
-  __nv_bfloat16 *kc, *vc;
+  __half *kc, *vc;  // bf16 values in the fp16 encoding
   int* len;
   void* ws;
   size_t ws_bytes;
   int* status;
   float* h;
-  __nv_bfloat16 *xn, *qbuf, *attn, *act, *blk_k, *blk_v;
+  __nv_bfloat16 *xn, *attn, *act;  // [2][rows][cols]: hi plane, lo plane at + *_lo elements
+  size_t xn_lo, attn_lo, act_lo;
+  __half *qbuf, *blk_k, *blk_v;
   float2* rope;
   unsigned long long* amax;
   int *draft_ids, *ar_ids;
@@ -300,10 +318,10 @@ WsLayout ws_layout(const orthrus_config* c, int B, int max_block, int max_rows_r
   };
   w.status = take(256);
   w.h = take((size_t)max_rows * D * 4);
-  w.xn = take((size_t)max_rows * D * 2);
+  w.xn = take((size_t)2 * max_rows * D * 2);  // hi and lo planes
   w.qbuf = take((size_t)max_rows * Hd * 2 + 128 * d * 2);
-  w.attn = take((size_t)max_rows * Hd * 2);
-  w.act = take((size_t)max_rows * F * 2);
+  w.attn = take((size_t)2 * max_rows * Hd * 2);
+  w.act = take((size_t)2 * max_rows * F * 2);
   w.rope = take((size_t)max_rows * (d / 2) * 8);
   w.amax = take((size_t)max_rows * 8);
   w.draft_ids = take((size_t)B * max_block * 4);
@@ -335,6 +353,22 @@ bool set_smem_attr(F* kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
+// The dynamic shared-memory opt-in is a property of (kernel, device): it is set once per
+// pair, under a lock, so that host threads and calls on a second GPU each get it.
+template <typename F>
+bool ensure_smem_attr(F* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<int, const void*>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const std::pair<int, const void*> key(dev, (const void*)kernel);
+  std::lock_guard<std::mutex> lock(mu);
+  if (std::find(done.begin(), done.end(), key) != done.end()) return true;
+  if (!set_smem_attr(kernel, bytes)) return false;
+  done.push_back(key);
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // launches
 // ---------------------------------------------------------------------------
@@ -351,12 +385,12 @@ cudaError_t launch_gemm(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs
   a.k_chunks = Kd / 64;
   a.total_units = (long long)a.m_tiles * a.n_tiles * a.k_chunks;
   const int G = (int)std::min<long long>(num_sms(), a.total_units);
-  const size_t fixed = gemm_smem_bytes(a.Mt, 0);
-  const size_t stage = 16384 + (size_t)a.Mt * 128;
+  a.planes = std::max(1, a.planes);
+  const size_t fixed = gemm_smem_bytes(a.Mt, 0, a.planes);
+  const size_t stage = 16384 + (size_t)a.Mt * 128 * a.planes;
   a.stages = (int)std::min<size_t>(12, (kSmemLimit - fixed) / stage);
-  const size_t smem = gemm_smem_bytes(a.Mt, a.stages);
-  static bool attr = false;
-  if (!attr) attr = set_smem_attr(gemm_kernel<EPI>, kSmemLimit);
+  const size_t smem = gemm_smem_bytes(a.Mt, a.stages, a.planes);
+  if (!ensure_smem_attr(gemm_kernel<EPI>, kSmemLimit)) return cudaErrorInvalidValue;
   return launch(gemm_kernel<EPI>, dim3(G), dim3(kGemmThreads), smem, st, tmW, tmX, a);
 }
 
@@ -365,12 +399,10 @@ cudaError_t launch_attention(int d, const CUtensorMap& tq, const CUtensorMap& tk
   dim3 grid(a.max_chunks, a.row_tiles, a.B * a.Hkv);
   const size_t smem = attn_smem_bytes(d);
   if (d == 128) {
-    static bool attr = false;
-    if (!attr) attr = set_smem_attr(attention_kernel<128>, kSmemLimit);
+    if (!ensure_smem_attr(attention_kernel<128>, kSmemLimit)) return cudaErrorInvalidValue;
     return launch(attention_kernel<128>, grid, dim3(kAttnThreads), smem, st, tq, tk, tv, tkb, tvb, a);
   } else {
-    static bool attr = false;
-    if (!attr) attr = set_smem_attr(attention_kernel<64>, kSmemLimit);
+    if (!ensure_smem_attr(attention_kernel<64>, kSmemLimit)) return cudaErrorInvalidValue;
     return launch(attention_kernel<64>, grid, dim3(kAttnThreads), smem, st, tq, tk, tv, tkb, tvb, a);
   }
 }
@@ -396,35 +428,26 @@ GemmArgs base_gemm_args(const Plan* P) {
   a.partial = P->gemm_part;
   a.tile_counter = P->gemm_cnt;
   a.status = P->status;
+  a.planes = 2;  // layer projections read both activation planes
   return a;
 }
 
 // ---------------------------------------------------------------------------
 // persistent forward kernel (draft and verify views, at most 128 token rows)
 // ---------------------------------------------------------------------------
-// ORTHRUS_PERSISTENT=0 in the environment selects the per-op kernels instead.
-bool persistent_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("ORTHRUS_PERSISTENT");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
-}
-
-int env_int(const char* name, int dflt) {
-  const char* e = getenv(name);
-  return e && *e ? atoi(e) : dflt;
+// Blocks whose token rows fit two ring stages (at most 96 rows at head_dim 128) run through
+// it; larger blocks take the per-op kernels.
+bool fwd_rows_fit(int M, int d) {
+  return M <= 128 && fwd_fixed_smem(d) + 2 * fwd_stage_bytes(round_up(M, 16)) <= kSmemLimit;
 }
 
 bool persistent_ok(const Plan* P, int Q) {
-  return persistent_enabled() && P->mega_slots > 0 && P->B * Q <= 128 && Q <= P->max_block + 1;
+  return P->mega_slots > 0 && fwd_rows_fit(P->B * Q, P->cfg.head_dim) && Q <= P->max_block + 1;
 }
 
 template <int D, bool TL, bool G2>
 cudaError_t launch_forward_inst(cudaLaunchConfig_t& cfg, const FwdArgs& a) {
-  static bool set = false;
-  if (!set) set = set_smem_attr(forward_kernel<D, TL, G2>, kSmemLimit);
+  if (!ensure_smem_attr(forward_kernel<D, TL, G2>, kSmemLimit)) return cudaErrorInvalidValue;
   return cudaLaunchKernelEx(&cfg, forward_kernel<D, TL, G2>, a);
 }
 
@@ -466,15 +489,15 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   // such boxes measured fastest at 4; deeper rings put more requests in flight than HBM
   // serves efficiently
   a.stages = (int)std::min<size_t>(4, (kSmemLimit - fwd_fixed_smem(a.d)) / stage);
-  a.stages = std::max(2, std::min(a.stages, env_int("ORTHRUS_STAGES", a.stages)));
+  a.stages = std::max(2, a.stages);
   const size_t smem = fwd_fixed_smem(a.d) + (size_t)a.stages * stage;
   a.cap = P->cap;
   a.max_block = P->max_block;
   a.batch = P->B;
   const int sms = num_sms();
   a.ck = P->fwd_ck;
-  a.lookahead = std::max(0, env_int("ORTHRUS_LOOKAHEAD", 2));  // 2 k-pair tiles measured best
-  a.poll_ns = std::max(0, env_int("ORTHRUS_POLL_NS", 64));
+  a.lookahead = 2;  // k-pair tiles of run-ahead past an unmet dependency: 2 measured best
+  a.poll_ns = 64;   // sleep between polls of a phase counter
   a.pending = pending;
   a.draft_ids = draft;
   a.len = P->len;
@@ -489,6 +512,9 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.qbuf = P->qbuf;
   a.attn = P->attn;
   a.act = P->act;
+  a.xg_lo = P->xn_lo;
+  a.attn_lo = P->attn_lo;
+  a.act_lo = P->act_lo;
   a.rope = P->rope;
   a.ss = P->ss;
   a.ss_ld = P->ss_ld;
@@ -584,6 +610,7 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
   aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
   aa.len = P->len;
   aa.out = P->attn;
+  aa.out_lo = P->attn_lo;
   aa.part_o = P->att_o;
   aa.part_ml = P->att_ml;
   aa.counter = P->att_cnt;
@@ -593,8 +620,8 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
   for (int l = 0; l < P->L; ++l) {
     const LayerPtrs& lp = P->layer(l);
     mark(P, ORTHRUS_KIND_RMSNORM, st);
-    if (launch(rmsnorm_kernel, dim3(M), dim3(256), 0, st, (const float*)P->h, D, lp.attn_norm, c.rms_eps, P->xn, 0, 1,
-               (unsigned long long*)nullptr) != cudaSuccess)
+    if (launch(rmsnorm_kernel, dim3(M), dim3(256), 0, st, (const float*)P->h, D, lp.attn_norm, c.rms_eps, P->xn,
+               P->xn_lo, 0, 1, (unsigned long long*)nullptr) != cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
     GemmArgs g = base_gemm_args(P);
@@ -624,7 +651,7 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
     }
     const int qkv_rows = (H + 2 * Hkv) * d;
     mark(P, ORTHRUS_KIND_GEMM_QKV, st);
-    if ((launch_gemm<EPI_QKV>(P->lmap(l, draft_view ? M_WDQKV : M_WQKV), P->gmap(G_XN + mt_index(M)), g, qkv_rows, D, M, st)) !=
+    if ((launch_gemm<EPI_QKV>(P->lmap(l, draft_view ? M_WDQKV : M_WQKV), P->gmap(G_XNP + mt_index(M)), g, qkv_rows, D, M, st)) !=
         cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
@@ -644,15 +671,16 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
       return ORTHRUS_ERR_CUDA;
 
     mark(P, ORTHRUS_KIND_RMSNORM, st);
-    if (launch(rmsnorm_kernel, dim3(M), dim3(256), 0, st, (const float*)P->h, D, lp.mlp_norm, c.rms_eps, P->xn, 0, 1,
-               (unsigned long long*)nullptr) != cudaSuccess)
+    if (launch(rmsnorm_kernel, dim3(M), dim3(256), 0, st, (const float*)P->h, D, lp.mlp_norm, c.rms_eps, P->xn,
+               P->xn_lo, 0, 1, (unsigned long long*)nullptr) != cudaSuccess)
       return ORTHRUS_ERR_CUDA;
     g = base_gemm_args(P);
     g.out_bf16 = P->act;
+    g.out_lo = P->act_lo;
     g.ld_out = F;
     g.swiglu_F = F;
     mark(P, ORTHRUS_KIND_GEMM_GATE_UP, st);
-    if ((launch_gemm<EPI_SWIGLU>(P->lmap(l, M_WGU), P->gmap(G_XN + mt_index(M)), g, 2 * F, D, M, st)) != cudaSuccess)
+    if ((launch_gemm<EPI_SWIGLU>(P->lmap(l, M_WGU), P->gmap(G_XNP + mt_index(M)), g, 2 * F, D, M, st)) != cudaSuccess)
       return ORTHRUS_ERR_CUDA;
 
     g = base_gemm_args(P);
@@ -667,9 +695,10 @@ orthrus_status forward(const Plan* P, int kind, int b0, int nb, int Q, const int
   const int HR = last_row_only ? nb : M;
   mark(P, ORTHRUS_KIND_RMSNORM, st);
   if (launch(rmsnorm_kernel, dim3(HR), dim3(256), 0, st, (const float*)P->h, D, P->final_norm, c.rms_eps, P->xn,
-             last_row_only ? Q - 1 : 0, last_row_only ? Q : 1, P->amax) != cudaSuccess)
+             (size_t)0, last_row_only ? Q - 1 : 0, last_row_only ? Q : 1, P->amax) != cudaSuccess)
     return ORTHRUS_ERR_CUDA;
   GemmArgs g = base_gemm_args(P);
+  g.planes = 1;  // the LM head reads the hi plane only
   g.amax = P->amax;
   g.logits = logits;
   g.ld_logits = V;
@@ -750,8 +779,8 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->embed = w->embed;
   P->final_norm = w->final_norm;
   P->lm_head = w->lm_head;
-  P->kc = (__nv_bfloat16*)cache->k;
-  P->vc = (__nv_bfloat16*)cache->v;
+  P->kc = (__half*)cache->k;
+  P->vc = (__half*)cache->v;
   P->len = cache->len;
   P->ws = workspace;
   P->ws_bytes = workspace_bytes;
@@ -759,9 +788,15 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->status = (int*)(base + wl.status);
   P->h = (float*)(base + wl.h);
   P->xn = (__nv_bfloat16*)(base + wl.xn);
-  P->qbuf = (__nv_bfloat16*)(base + wl.qbuf);
+  P->qbuf = (__half*)(base + wl.qbuf);
   P->attn = (__nv_bfloat16*)(base + wl.attn);
   P->act = (__nv_bfloat16*)(base + wl.act);
+  {
+    const size_t r = (size_t)act_rows(max_rows);
+    P->xn_lo = r * cfg->d_model;
+    P->attn_lo = r * cfg->n_heads * cfg->head_dim;
+    P->act_lo = r * cfg->d_ff;
+  }
   P->rope = (float2*)(base + wl.rope);
   P->amax = (unsigned long long*)(base + wl.amax);
   P->draft_ids = (int*)(base + wl.draft_ids);
@@ -773,8 +808,8 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->att_o = (float*)(base + wl.att_o);
   P->att_ml = (float2*)(base + wl.att_ml);
   P->att_cnt = (int*)(base + wl.att_cnt);
-  P->blk_k = (__nv_bfloat16*)(base + wl.blk_k);
-  P->blk_v = (__nv_bfloat16*)(base + wl.blk_v);
+  P->blk_k = (__half*)(base + wl.blk_k);
+  P->blk_v = (__half*)(base + wl.blk_v);
   P->d_maps = (CUtensorMap*)(base + wl.dev_maps);
   P->d_norms = (LayerNorms*)(base + wl.dev_norms);
   P->phase_cnt = (int*)(base + wl.phase_cnt);
@@ -784,7 +819,6 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->mega_slots = wl.mega_slots;
   // attention chunk of the persistent kernel: at most kMaxChunks - 2 chunks over the whole capacity
   P->fwd_ck = std::max(64, round_up((P->cap + kMaxChunks - 3) / (kMaxChunks - 2), 64));
-  P->fwd_ck = std::max(P->fwd_ck, round_up(env_int("ORTHRUS_ATT_CK", 0), 64));
   P->fwd_att_o = (float*)(base + wl.fwd_att_o);
   P->fwd_att_ml = (float2*)(base + wl.fwd_att_ml);
   P->norms_off = norms_off;
@@ -843,23 +877,26 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   ok = ok && map_kpair(P->gmap_mut(G_LM3), w->lm_head, D, V, 128);
   const int rows = act_rows(max_rows);
   for (int i = 0; i < 8; ++i) {
-    ok = ok && map2d(P->gmap_mut(G_XN + i), P->xn, D, rows, 64, 16 * (i + 1));
-    ok = ok && map2d(P->gmap_mut(G_ATTN + i), P->attn, H * d, rows, 64, 16 * (i + 1));
-    ok = ok && map2d(P->gmap_mut(G_ACT + i), P->act, F, rows, 64, 16 * (i + 1));
-    ok = ok && map_kpair(P->gmap_mut(G_XN3 + i), P->xn, D, rows, 16 * (i + 1));
-    ok = ok && map_kpair(P->gmap_mut(G_ATTN3 + i), P->attn, H * d, rows, 16 * (i + 1));
-    ok = ok && map_kpair(P->gmap_mut(G_ACT3 + i), P->act, F, rows, 16 * (i + 1));
+    const uint32_t br = 16 * (i + 1);
+    ok = ok && map2d(P->gmap_mut(G_XN + i), P->xn, D, rows, 64, br);  // hi plane only
+    ok = ok && map_planes(P->gmap_mut(G_XNP + i), P->xn, D, rows, br);
+    ok = ok && map_planes(P->gmap_mut(G_ATTN + i), P->attn, H * d, rows, br);
+    ok = ok && map_planes(P->gmap_mut(G_ACT + i), P->act, F, rows, br);
+    ok = ok && map_kpair(P->gmap_mut(G_XN3 + i), P->xn, D, rows, br);  // hi plane only
+    ok = ok && map_kpair_planes(P->gmap_mut(G_XN4 + i), P->xn, D, rows, br);
+    ok = ok && map_kpair_planes(P->gmap_mut(G_ATTN4 + i), P->attn, H * d, rows, br);
+    ok = ok && map_kpair_planes(P->gmap_mut(G_ACT4 + i), P->act, F, rows, br);
   }
-  ok = ok && map2d(P->gmap_mut(G_Q), P->qbuf, d, (uint64_t)rows * H + 128, 64, 128);
+  ok = ok && map2d(P->gmap_mut(G_Q), P->qbuf, d, (uint64_t)rows * H + 128, 64, 128, kF16);
   const uint64_t zc = (uint64_t)L * P->B * Hkv;
-  ok = ok && map3d(P->gmap_mut(G_KC), P->kc, d, P->cap, zc);
-  ok = ok && map3d(P->gmap_mut(G_VC), P->vc, d, P->cap, zc);
-  ok = ok && map3d(P->gmap_mut(G_KB), P->blk_k, d, max_block, zc);
-  ok = ok && map3d(P->gmap_mut(G_VB), P->blk_v, d, max_block, zc);
-  ok = ok && map3d(P->gmap_mut(G_KC64), P->kc, d, P->cap, zc, 64);
-  ok = ok && map3d(P->gmap_mut(G_VC64), P->vc, d, P->cap, zc, 64);
-  ok = ok && map3d(P->gmap_mut(G_KB64), P->blk_k, d, max_block, zc, 64);
-  ok = ok && map3d(P->gmap_mut(G_VB64), P->blk_v, d, max_block, zc, 64);
+  ok = ok && map3d(P->gmap_mut(G_KC), P->kc, d, P->cap, zc, 128, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_VC), P->vc, d, P->cap, zc, 128, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_KB), P->blk_k, d, max_block, zc, 128, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_VB), P->blk_v, d, max_block, zc, 128, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_KC64), P->kc, d, P->cap, zc, 64, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_VC64), P->vc, d, P->cap, zc, 64, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_KB64), P->blk_k, d, max_block, zc, 64, 1, kF16);
+  ok = ok && map3d(P->gmap_mut(G_VB64), P->blk_v, d, max_block, zc, 64, 1, kF16);
   if (!ok) return ORTHRUS_ERR_ARG;
   if (cudaMemsetAsync(workspace, 0, wl.total, (cudaStream_t)stream) != cudaSuccess) return ORTHRUS_ERR_CUDA;
   // the persistent kernel reads the tensor maps and norm gains from device memory
@@ -1196,9 +1233,12 @@ orthrus_status orthrus_attention(const void* q, const void* k_cache, const void*
   if (cudaMemsetAsync(counter, 0, slots * 4, st) != cudaSuccess) return ORTHRUS_ERR_CUDA;
   CUtensorMap tq, tk, tv, tkb, tvb;
   const uint64_t z = (uint64_t)batch * n_kv_heads;
-  bool ok = map2d(&tq, q, head_dim, z * Q * group, 64, 128);
-  ok = ok && map3d(&tk, k_cache, head_dim, capacity, z) && map3d(&tv, v_cache, head_dim, capacity, z);
-  if (mode == 0) ok = ok && map3d(&tkb, k_blk, head_dim, blk_stride, z) && map3d(&tvb, v_blk, head_dim, blk_stride, z);
+  bool ok = map2d(&tq, q, head_dim, z * Q * group, 64, 128, kF16);
+  ok = ok && map3d(&tk, k_cache, head_dim, capacity, z, 128, 1, kF16) &&
+       map3d(&tv, v_cache, head_dim, capacity, z, 128, 1, kF16);
+  if (mode == 0)
+    ok = ok && map3d(&tkb, k_blk, head_dim, blk_stride, z, 128, 1, kF16) &&
+         map3d(&tvb, v_blk, head_dim, blk_stride, z, 128, 1, kF16);
   else {
     tkb = tk;
     tvb = tv;
@@ -1223,6 +1263,7 @@ orthrus_status orthrus_attention(const void* q, const void* k_cache, const void*
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   a.len = len;
   a.out = (__nv_bfloat16*)out;
+  a.out_lo = (size_t)batch * Q * n_kv_heads * group * head_dim;
   a.part_o = part_o;
   a.part_ml = part_ml;
   a.counter = counter;
@@ -1309,12 +1350,12 @@ cudaError_t launch_gemm_capped(const CUtensorMap& tmW, const CUtensorMap& tmX, G
   a.k_chunks = Kd / 64;
   a.total_units = (long long)a.m_tiles * a.n_tiles * a.k_chunks;
   const int G = (int)std::min<long long>(std::min(num_sms(), max_ctas), a.total_units);
-  const size_t fixed = gemm_smem_bytes(a.Mt, 0);
+  a.planes = 1;  // the caller's X is one bf16 matrix
+  const size_t fixed = gemm_smem_bytes(a.Mt, 0, 1);
   const size_t stage = 16384 + (size_t)a.Mt * 128;
   a.stages = (int)std::min<size_t>(12, (kSmemLimit - fixed) / stage);
-  const size_t smem = gemm_smem_bytes(a.Mt, a.stages);
-  static bool attr = false;
-  if (!attr) attr = set_smem_attr(gemm_kernel<EPI>, kSmemLimit);
+  const size_t smem = gemm_smem_bytes(a.Mt, a.stages, 1);
+  if (!ensure_smem_attr(gemm_kernel<EPI>, kSmemLimit)) return cudaErrorInvalidValue;
   return launch(gemm_kernel<EPI>, dim3(G), dim3(kGemmThreads), smem, st, tmW, tmX, a);
 }
 }  // namespace

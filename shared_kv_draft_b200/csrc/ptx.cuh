@@ -7,6 +7,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "orthrus.h"
@@ -272,6 +273,14 @@ __device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
                                                  int w, uint64_t policy) {
   asm volatile(
@@ -323,8 +332,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16: bf16 or fp16 inputs (the instruction
+// descriptor names the type, the same for both operands), fp32 accumulate.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -422,6 +432,67 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Same with fp16 A and B (format 0): both operands of one MMA must have the same type.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// operand encodings
+// ---------------------------------------------------------------------------
+// An activation operand is carried as two bf16 planes, x = hi + lo with hi = bf16(x) and
+// lo = bf16(x - hi): about 16 significant bits. Both planes are multiplied by the same
+// bf16 weights and accumulated in fp32, so a projection sees x to about 2^-17 relative
+// instead of the 2^-9 of one bf16 rounding.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// 16 floats -> hi plane (16-byte aligned dst_hi) and lo plane (dst_lo), two 16-byte stores each
+__device__ __forceinline__ void st_split_x16(__nv_bfloat16* dst_hi, __nv_bfloat16* dst_lo, const float* x) {
+  uint32_t h[8], l[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) split_bf16x2(x[2 * i], x[2 * i + 1], h[i], l[i]);
+  uint4* ph = reinterpret_cast<uint4*>(dst_hi);
+  uint4* pl = reinterpret_cast<uint4*>(dst_lo);
+  ph[0] = make_uint4(h[0], h[1], h[2], h[3]);
+  ph[1] = make_uint4(h[4], h[5], h[6], h[7]);
+  pl[0] = make_uint4(l[0], l[1], l[2], l[3]);
+  pl[1] = make_uint4(l[4], l[5], l[6], l[7]);
+}
+
+// 8 floats -> one 16-byte store to each plane
+__device__ __forceinline__ void st_split_x8(__nv_bfloat16* dst_hi, __nv_bfloat16* dst_lo, const float* x) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) split_bf16x2(x[2 * i], x[2 * i + 1], h[i], l[i]);
+  *reinterpret_cast<uint4*>(dst_hi) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(dst_lo) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Attention operands are fp16: q and the softmax weights P carry 11 significant bits
+// (bf16: 8), and K and V, whose values are bf16 (the cache precision), are held in the
+// fp16 encoding so that one MMA sees one operand type. Every bf16 value of magnitude in
+// [2^-17, 65504] is an fp16 value; smaller ones round to the nearest fp16 (error < 2^-25).
+__device__ __forceinline__ float kv_value(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// 16 floats -> fp16, two 16-byte stores
+__device__ __forceinline__ void st_f16x16(__half* dst, const float* x) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __half2 h2 = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h2);
+  }
+  uint4* p = reinterpret_cast<uint4*>(dst);
+  p[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  p[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 // ---------------------------------------------------------------------------
 // small math helpers
 // ---------------------------------------------------------------------------
@@ -445,9 +516,12 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Order-preserving map of a (non-NaN) float to uint32.
+// Order-preserving map of a (non-NaN) float to uint32. -0.0 and +0.0 compare equal as
+// numbers, so both map to the key of +0.0: an exact tie between them then goes to the
+// lower index like any other tie.
 __device__ __forceinline__ uint32_t float_order_key(float f) {
   uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -1,6 +1,6 @@
 // Small kernels of the decode step: block embedding (+ RoPE table and the
-// capacity check), RMSNorm to bf16, argmax finalisation, greedy consensus with
-// the KV commit, and dead-slot poisoning.
+// capacity check), RMSNorm to bf16 hi/lo planes, argmax finalisation, greedy
+// consensus with the KV commit, and dead-slot poisoning.
 #pragma once
 #include "ptx.cuh"
 
@@ -66,9 +66,10 @@ __global__ void embed_kernel(const EmbedArgs a) {
   }
 }
 
-// out[m] = bf16( h[src_first + m*src_stride] * rsqrt(mean(h^2) + eps) * gain ); optionally zero keys[m]
+// x = h[src_first + m*src_stride] * rsqrt(mean(h^2) + eps) * gain -> out[m] = bf16(x), and with
+// out_lo > 0 also the lo plane out[out_lo + m] = bf16(x - bf16(x)); optionally zero keys[m]
 __global__ void rmsnorm_kernel(const float* __restrict__ h, int D, const float* __restrict__ gain, float eps,
-                               __nv_bfloat16* __restrict__ out, int src_first, int src_stride,
+                               __nv_bfloat16* __restrict__ out, size_t out_lo, int src_first, int src_stride,
                                unsigned long long* reset_keys) {
   griddep_wait();
   griddep_launch();
@@ -94,10 +95,11 @@ __global__ void rmsnorm_kernel(const float* __restrict__ h, int D, const float* 
   for (int c = threadIdx.x * 4; c < D; c += blockDim.x * 4) {
     const float4 v = *reinterpret_cast<const float4*>(x + c);
     const float4 g = *reinterpret_cast<const float4*>(gain + c);
-    __nv_bfloat162 a0 = __floats2bfloat162_rn(v.x * r * g.x, v.y * r * g.y);
-    __nv_bfloat162 a1 = __floats2bfloat162_rn(v.z * r * g.z, v.w * r * g.w);
-    uint2 pk = make_uint2(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1));
-    *reinterpret_cast<uint2*>(y + c) = pk;
+    uint32_t h0, h1, l0, l1;
+    split_bf16x2(v.x * r * g.x, v.y * r * g.y, h0, l0);
+    split_bf16x2(v.z * r * g.z, v.w * r * g.w, h1, l1);
+    *reinterpret_cast<uint2*>(y + c) = make_uint2(h0, h1);
+    if (out_lo) *reinterpret_cast<uint2*>(y + out_lo + c) = make_uint2(l0, l1);
   }
   if (reset_keys && threadIdx.x == 0) reset_keys[m] = 0ull;
 }
@@ -155,8 +157,8 @@ __global__ void accept_kernel(int* pending, const int* draft, const int* ar, int
 }
 
 // Overwrite the dead verify slots [len, len + K - a) of every layer and KV head
-// with NaN (bf16 0x7FC0), after accept_kernel advanced len.
-__global__ void poison_kernel(__nv_bfloat16* kc, __nv_bfloat16* vc, const int* len, const int* accept_len, int K,
+// with NaN (fp16 0x7E00), after accept_kernel advanced len.
+__global__ void poison_kernel(__half* kc, __half* vc, const int* len, const int* accept_len, int K,
                               int B, int Hkv, int cap, int d) {
   griddep_wait();
   griddep_launch();
@@ -165,7 +167,7 @@ __global__ void poison_kernel(__nv_bfloat16* kc, __nv_bfloat16* vc, const int* l
   const int a = accept_len[b];
   if (a < 0) return;
   const int lo = len[b], hi = min(cap, len[b] + K - a);
-  const __nv_bfloat16 nan = __ushort_as_bfloat16((unsigned short)0x7FC0);
+  const __half nan = __ushort_as_half((unsigned short)0x7E00);
   for (int s = lo; s < hi; ++s) {
     for (int e = threadIdx.x; e < d; e += blockDim.x) {
       kc[((size_t)z * cap + s) * d + e] = nan;

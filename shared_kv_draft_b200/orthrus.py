@@ -53,9 +53,14 @@ class Cache(C.Structure):
                 ("capacity", C.c_int32)]
 
 
+class AcceptStats(C.Structure):
+    _fields_ = [("accepted", C.c_float), ("rejected", C.c_float)]
+
+
 # (name, restype, argtypes) for every symbol of include/orthrus.h
 _I32, _SZ, _VP, _F = C.c_int32, C.c_size_t, C.c_void_p, C.c_float
 _PCFG = C.POINTER(Config)
+_PST = C.POINTER(AcceptStats)
 SIGNATURES = [
     ("orthrus_plan_bytes", _SZ, [_PCFG]),
     ("orthrus_workspace_bytes", _SZ, [_PCFG, _I32, _I32, _I32, _I32]),
@@ -84,6 +89,9 @@ SIGNATURES = [
     ("orthrus_linear_workspace_bytes", _SZ, [_I32, _I32, _I32]),
     ("orthrus_linear", _I32, [_VP, _VP, _VP, _I32, _I32, _I32, _VP, _SZ, _VP, _VP]),
     ("orthrus_linear_noalloc", _I32, [_VP, _VP, _VP, _I32, _I32, _I32, _VP, _VP]),
+    ("orthrus_accept_stats_update", _I32, [_PST, _VP, _I32, _I32, _F]),
+    ("orthrus_accept_rate", _F, [_PST]),
+    ("orthrus_choose_block_size", _I32, [_PST, _I32, _VP, _VP, _I32]),
 ]
 
 _lib = None
@@ -148,6 +156,7 @@ def block_scratch_offset(cfg: Config, batch: int, capacity: int, max_block: int,
 
 def attention(q, k_cache, v_cache, k_blk, v_blk, lens, batch, n_kv_heads, group, Q, head_dim, capacity, blk_stride,
               mode, out, workspace, status, stream=None):
+    """q, K and V in fp16 (device); out: bf16 [2][batch * Q][heads * head_dim], hi then lo plane."""
     lib = load()
     code = lib.orthrus_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_blk), _ptr(v_blk), _ptr(lens), batch,
                                  n_kv_heads, group, Q, head_dim, capacity, blk_stride, mode, _ptr(out),
@@ -186,6 +195,33 @@ def sample_tokens(logits, temperature, uniforms, out, status=None, stream=None):
     _check("orthrus_sample_tokens", code)
 
 
+def accept_stats(batch: int):
+    """Zeroed acceptance counts of `batch` sequences (host memory)."""
+    return (AcceptStats * batch)()
+
+
+def accept_stats_update(stats, accept_len, K: int, decay: float = 1.0):
+    """Fold one step's host accept lengths (ints) into `stats`."""
+    n = len(accept_len)
+    arr = (C.c_int32 * n)(*[int(a) for a in accept_len])
+    _check("orthrus_accept_stats_update", load().orthrus_accept_stats_update(stats, arr, n, K, float(decay)))
+
+
+def accept_rate(stats, b: int = 0) -> float:
+    return float(load().orthrus_accept_rate(C.byref(stats[b])))
+
+
+def choose_block_size(stats, ks, step_ms) -> int:
+    """The K of `ks` that commits the most tokens per ms (measured step times `step_ms`)."""
+    n = len(ks)
+    k_arr = (C.c_int32 * n)(*[int(k) for k in ks])
+    t_arr = (C.c_float * n)(*[float(t) for t in step_ms])
+    k = load().orthrus_choose_block_size(stats, len(stats), k_arr, t_arr, n)
+    if k < 0:
+        raise OrthrusError("orthrus_choose_block_size", ERR_ARG)
+    return int(k)
+
+
 def linear_workspace_bytes(M, N, Kd) -> int:
     return load().orthrus_linear_workspace_bytes(M, N, Kd)
 
@@ -220,7 +256,8 @@ class DeviceModel:
         self.cfg = make_config(shape)
         self.dev = {k: (v if isinstance(v, torch.Tensor) else upload(v, device)) for k, v in weights.items()}
         L, Hkv, d = shape.n_layers, shape.n_kv_heads, shape.head_dim
-        self.k_cache = torch.zeros((L, batch, Hkv, capacity, d), dtype=torch.bfloat16, device=device)
+        # K/V cache: bf16 values held in the fp16 encoding (the attention MMAs take fp16 operands)
+        self.k_cache = torch.zeros((L, batch, Hkv, capacity, d), dtype=torch.float16, device=device)
         self.v_cache = torch.zeros_like(self.k_cache)
         self.lens = torch.zeros(batch, dtype=torch.int32, device=device)
         self._arrays = {}

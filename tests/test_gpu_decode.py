@@ -300,11 +300,14 @@ def test_large_batch_per_op_path_matches_oracle():
     print(stats)
 
 
-@pytest.mark.parametrize("B,K", [(1, 33), (4, 8), (2, 17)], ids=["rows34", "rows36", "rows36_b2"])
+@pytest.mark.parametrize("B,K", [(1, 33), (4, 8), (2, 17), (2, 32), (3, 24), (4, 16), (1, 64)],
+                         ids=["rows34", "rows36", "rows36_b2", "rows66", "rows75", "rows68", "rows65"])
 def test_token_rows_past_32_match_oracle(B, K):
-    """Verify blocks of 34-36 token rows: the projections' epilogues handle a second group
-    of token columns past the first 32 (the 33rd row of a K = 32 verify block). Draft and
-    verify logits and argmaxes of every sequence match the oracle."""
+    """Blocks of 34-96 token rows on the persistent kernel: the projections' epilogues handle
+    a second group of token columns past the first 32 (the 33rd row of a K = 32 verify
+    block) and further 32-row groups, including split tiles with several rounds of
+    contributors (the tiny model's down projection splits each tile over six CTAs). Draft
+    and verify logits and argmaxes of every sequence match the oracle."""
     shape = synth.TINY_QK
     rng = np.random.default_rng(90 + B)
     lens = rng.integers(10, 40, size=B).tolist()

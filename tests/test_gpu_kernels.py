@@ -56,6 +56,10 @@ def test_linear_matches_oracle(M, N, Kd):
 
 
 def run_attention(B, Hkv, G, Q, d, cap, lens, mode, seed, poison=False, blk_stride=None):
+    """Block attention through orthrus_attention against the oracle. q, K and V are bf16
+    values (N(0, 1) from a seed); the kernel takes them in the fp16 encoding, which holds
+    every such value of magnitude >= 2^-17 exactly, and writes the output as two bf16
+    planes (hi, lo) whose sum is compared."""
     o = lib()
     H = Hkv * G
     blk_stride = blk_stride or Q
@@ -72,15 +76,16 @@ def run_attention(B, Hkv, G, Q, d, cap, lens, mode, seed, poison=False, blk_stri
             vc[b, :, live:] = nan
             kb[b, :, Q:] = nan
             vb[b, :, Q:] = nan
-    out = torch.full((B, Q, H * d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    f16 = lambda t: t.to(torch.float16).cuda()
+    out = torch.full((2, B, Q, H * d), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(o.attention_workspace_bytes(B, Hkv, G, Q, d, cap), dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     ln = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    o.attention(q.cuda(), kc.cuda(), vc.cuda(), kb.cuda(), vb.cuda(), ln, B, Hkv, G, Q, d, cap, blk_stride, mode, out,
+    o.attention(f16(q), f16(kc), f16(vc), f16(kb), f16(vb), ln, B, Hkv, G, Q, d, cap, blk_stride, mode, out,
                 ws, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    got = out.float().cpu().numpy()
+    got = (out[0].double() + out[1].double()).cpu().numpy()
     for b in range(B):
         n = lens[b]
         qo = q[b].to(torch.float64).reshape(Hkv, Q, G, d).permute(1, 0, 2, 3).reshape(Q, H, d)

@@ -1,53 +1,145 @@
-"""GPU runs at the two large workload shapes of the Qwen3-8B-shaped model, checked by
-properties that hold at any size (the fp64 oracle cannot prefill thousands of tokens
-through 36 layers within a test):
+"""GPU runs at the two large workload shapes of the Qwen3-8B-shaped model:
+  - config 4: batch 16 with ragged cache lengths uniform in [1024, 8192], K = 32;
+  - config 5: batch 4 at a 32768-token cache, K in {8, 16, 32, 64}.
+Blocks of at most 96 token rows run through the persistent kernel, larger ones through
+the per-op kernels (config 4's 512/528-row blocks; config 5 at K = 32 and 64).
 
-- batch 16 with ragged cache lengths uniform in [1024, 8192], K = 32: the 528-row verify
-  blocks run through the per-op kernels, the plain-AR steps through the persistent kernel;
-- batch 4 at a 32768-token cache, K = 8 (persistent kernel) and K = 64 (per-op kernels).
+Two kinds of checks (the fp64 oracle cannot prefill tens of thousands of tokens through
+36 layers within a test):
 
-Each sequence's greedy AR stream is built on the GPU first (verify with K = 0, one token per
-forward, the commit after it). The cache lengths and pending tokens are then put back to
-their post-prefill values (slots past a length are dead and every forward overwrites them
-before reading), and one step runs on planted drafts: the first a tokens of the greedy
-stream, then a token that differs from it, then uniform ids (draft, verify with logits,
-accept/commit). Checked:
-- bit-exact: the accept length is the first draft that differs from the AR argmax, the
-  committed ids are those drafts and the AR token, the cache length advances by a + 1, the
-  pending token is the AR token, the status word stays clear;
-- every verify row whose inputs are the greedy prefix returns the greedy token, or the
-  greedy token's logit is within 0.1 of the row's maximum (the margin rule: kernels that
-  round differently may resolve a near tie differently). When the verify rows go through
-  the persistent kernel, as the AR rows do, they are bit-identical and no row differs;
-- with no such near tie, the accept length equals the planted one.
-Attention over a 32768-token cache is also compared with the oracle (one layer).
-Weights: seeded N(0, 0.02) bf16 drawn on the device; prompts: seeded uniform ids.
+1. Oracle parity on sampled sequences. The cache of the sampled sequences holds seeded
+   synthetic K/V (N(0, 1) keys, as after QK-RMSNorm, and N(0, 1.28^2) values, the scale
+   of x W_v for unit-RMS x and N(0, 0.02) weights), written into the library's cache and
+   into the oracle's: the same bf16 values on both sides, none from the GPU. One draft
+   and one verify forward on seeded random drafts then run on the GPU for the whole batch;
+   the oracle recomputes the sampled sequences. Draft and verify logits within max-abs
+   5e-2, tokens bit-exact where the oracle's top-2 margin > 0.1 (else within 0.1 of its
+   maximum), the consensus on the GPU's drafts and argmaxes bit-exact.
+2. Properties at full size after a real prefill: each sequence's greedy AR stream is
+   built on the GPU (verify with K = 0); one step on drafts planted from it must then
+   commit exactly the planted prefix and the AR token (rows resolved differently only
+   at near ties, within the margin rule), with cache lengths and pending tokens exact.
+Attention over a 32768-token cache is also compared with the oracle alone (one layer).
 """
 import numpy as np
 import pytest
 import torch
 
 import synth
+from oracle import Oracle, accept_length, top2_margin
 
 pytestmark = pytest.mark.gpu
 
+MARGIN = 0.1
+LOGIT_TOL = 5e-2
+V_STD = 1.28  # std of x W_v: sqrt(4096) * 0.02
 
-def device_weights(shape, seed):
+
+def bf16_to_f16_dev(bits):
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda().to(torch.float16)
+
+
+def fill_synthetic_cache(dev, o_states, shape, lens, sampled, seed):
+    """Seeded K/V for positions [0, lens[b]) of every layer: sampled sequences get host-drawn
+    bf16 values (also loaded into their oracle states); the others get device-drawn ones."""
+    L, Hkv, d = shape.n_layers, shape.n_kv_heads, shape.head_dim
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
-    w = {}
-    for name, dims, kind in synth.tensor_specs(shape):
-        if kind == "gain":
-            w[name] = torch.ones(dims, dtype=torch.float32, device="cuda")
+    for b, n in enumerate(lens):
+        if b in sampled:
+            kb = synth.normal_bf16((L, Hkv, n, d), seed + 10 * b + 1)
+            vb = synth.normal_bf16((L, Hkv, n, d), seed + 10 * b + 2, std=V_STD)
+            dev.k_cache[:, b, :, :n] = bf16_to_f16_dev(kb)
+            dev.v_cache[:, b, :, :n] = bf16_to_f16_dev(vb)
+            st = o_states[b]
+            kt = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16)
+            vt = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16)
+            for l in range(L):
+                st.k[l][:, :n] = kt[l]
+                st.v[l][:, :n] = vt[l]
+            st.n = n
         else:
-            w[name] = (torch.randn(dims, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
-    return w
+            for l in range(L):
+                kx = torch.randn((Hkv, n, d), generator=g, device="cuda")
+                vx = torch.randn((Hkv, n, d), generator=g, device="cuda") * V_STD
+                dev.k_cache[l, b, :, :n] = kx.to(torch.bfloat16).to(torch.float16)
+                dev.v_cache[l, b, :, :n] = vx.to(torch.bfloat16).to(torch.float16)
+    dev.lens.copy_(torch.tensor(lens, dtype=torch.int32))
 
 
-MARGIN = 0.1
+def follow(tok, row):
+    best = int(torch.argmax(row))
+    if top2_margin(row) > MARGIN:
+        assert tok == best, (tok, best)
+        return 0
+    assert float(row[tok]) >= float(row[best]) - MARGIN, (tok, best)
+    return 1
 
 
-def run_property_check(B, lens, K, mean_accept, seed):
+def check_logits(gpu, ref, what):
+    err = float(np.abs(gpu - ref.numpy()).max())
+    print(f"  {what}: max-abs {err:.4f}")
+    assert err <= LOGIT_TOL, (what, err)
+
+
+def run_oracle_sampled(qwen_host_weights, qwen_device_weights, lens, Ks, sampled, seed):
+    from shared_kv_draft_b200 import orthrus
+    shape = synth.QWEN3_8B
+    B, V = len(lens), shape.vocab
+    Kmax = max(Ks)
+    cap = max(lens) + Kmax + 8
+    dev = orthrus.DeviceModel(shape, qwen_device_weights, batch=B, capacity=cap, max_block=Kmax,
+                              max_rows=max(64, B * (Kmax + 1)))
+    o = Oracle(shape, qwen_host_weights, capacity=cap)
+    states = {b: o.new_state() for b in sampled}
+    fill_synthetic_cache(dev, states, shape, lens, sampled, seed)
+    rng = np.random.default_rng(seed + 1)
+    pend_h = rng.integers(0, V, size=B).astype(np.int32)
+    near = 0
+    for K in Ks:
+        z = lambda *s: torch.zeros(s, dtype=torch.int32, device="cuda")
+        pending = torch.from_numpy(pend_h).cuda()
+        planted = rng.integers(0, V, size=(B, K)).astype(np.int32)
+        drafts = torch.from_numpy(planted).cuda()
+        dout, ar, acc, com = z(B, K), z(B, K + 1), z(B), z(B, K + 1)
+        dlog = torch.zeros((B, K, V), device="cuda")
+        vlog = torch.zeros((B, K + 1, V), device="cuda")
+        dev.draft_block(pending, K, dout, dlog)
+        dev.verify_block(pending, drafts, K, ar, vlog)
+        dev.accept_commit(pending, drafts, ar, K, acc, com)
+        torch.cuda.synchronize()
+        assert dev.read_status() == 0
+        print(f"batch {B}, K = {K}:")
+        arh, dh = ar.cpu().numpy(), dout.cpu().numpy()
+        for b in range(B):  # consensus of every sequence on its drafts and AR argmaxes: bit-exact
+            a = accept_length(planted[b].tolist(), arh[b].tolist())
+            assert int(acc[b]) == a and com[b, :a + 1].cpu().tolist() == planted[b, :a].tolist() + [int(arh[b, a])]
+            assert int(dev.lens[b]) == lens[b] + a + 1
+        dev.lens.copy_(torch.tensor(lens, dtype=torch.int32))  # back to the synthetic cache for the next K
+        for b in sampled:
+            st = states[b]
+            st.y = int(pend_h[b])
+            _, dl = o.draft_block(st, K)
+            check_logits(dlog[b].cpu().numpy(), dl, f"seq {b} (cache {lens[b]}) draft logits")
+            near += sum(follow(int(t), dl[i]) for i, t in enumerate(dh[b]))
+            _, vl = o.verify_block(st, planted[b].tolist())
+            check_logits(vlog[b].cpu().numpy(), vl, f"seq {b} verify logits")
+            near += sum(follow(int(t), vl[j]) for j, t in enumerate(arh[b]))
+    print(f"tokens within the 0.1 margin: {near}")
+
+
+def test_config4_batch16_ragged_matches_oracle_on_sampled_sequences(qwen_host_weights, qwen_device_weights):
+    rng = np.random.default_rng(41)
+    lens = rng.integers(1024, 8193, size=16).tolist()
+    sampled = [int(np.argmin(lens)), int(np.argmax(lens))]
+    run_oracle_sampled(qwen_host_weights, qwen_device_weights, lens, [32], sampled, seed=410)
+
+
+def test_config5_batch4_32k_matches_oracle_on_a_sampled_sequence(qwen_host_weights, qwen_device_weights):
+    run_oracle_sampled(qwen_host_weights, qwen_device_weights, [32768] * 4, [8, 16, 32, 64], [1], seed=500)
+
+
+def run_property_check(qwen_device_weights, B, lens, K, mean_accept, seed):
     from shared_kv_draft_b200 import orthrus
 
     shape = synth.QWEN3_8B
@@ -55,14 +147,14 @@ def run_property_check(B, lens, K, mean_accept, seed):
     accepts = np.array([synth.planted_accepts(1, mean_accept, K, seed=seed + b)[0] for b in range(B)])
     need = int(np.max(accepts)) + K + 3  # greedy tokens the planted drafts read
     cap = ((max(lens) + need + K + 2 + 127) // 128) * 128
-    w = device_weights(shape, seed)
-    dev = orthrus.DeviceModel(shape, w, batch=B, capacity=cap, max_block=K, max_rows=max(B * (K + 1), 512))
-    g = torch.Generator(device="cuda")
-    g.manual_seed(seed + 100)
-    toks = torch.randint(0, V, (B, max(lens)), generator=g, device="cuda", dtype=torch.int32)
+    dev = orthrus.DeviceModel(shape, qwen_device_weights, batch=B, capacity=cap, max_block=K,
+                              max_rows=max(B * (K + 1), 512))
+    toks = np.zeros((B, max(lens)), dtype=np.int32)
+    for b, n in enumerate(lens):
+        toks[b, :n] = synth.make_prompt(shape, n, seed + 100 + b)
     z = lambda *s: torch.zeros(s, dtype=torch.int32, device="cuda")
     pending = z(B)
-    dev.prefill(toks, lens, pending)
+    dev.prefill(torch.from_numpy(toks).cuda(), lens, pending)
     torch.cuda.synchronize()
     assert dev.read_status() == 0
     lens0 = dev.lens.clone()
@@ -122,16 +214,16 @@ def run_property_check(B, lens, K, mean_accept, seed):
     return flips
 
 
-def test_batch16_ragged_1k_to_8k_k32():
+def test_batch16_ragged_1k_to_8k_k32(qwen_device_weights):
     rng = np.random.default_rng(41)
     lens = rng.integers(1024, 8193, size=16).tolist()
-    run_property_check(16, lens, 32, 6.0, seed=41)
+    run_property_check(qwen_device_weights, 16, lens, 32, 6.0, seed=41)
 
 
-@pytest.mark.parametrize("K", [8, 64])
-def test_batch4_32k_cache(K):
-    flips = run_property_check(4, [32768] * 4, K, K / 5.0, seed=50 + K)
-    if 4 * (K + 1) <= 128:  # verify rows through the persistent kernel, like the AR rows: bit-identical
+@pytest.mark.parametrize("K", [8, 16, 32, 64])
+def test_batch4_32k_cache(qwen_device_weights, K):
+    flips = run_property_check(qwen_device_weights, 4, [32768] * 4, K, K / 5.0, seed=50 + K)
+    if 4 * (K + 1) <= 96:  # verify rows through the persistent kernel, like the AR rows: bit-identical
         assert flips == 0
 
 

@@ -1,120 +1,148 @@
 """GPU parity at the full Qwen3-8B shape (36 layers, hidden 4096, 32/8 heads, head_dim
-128, QK-norm, SwiGLU 12288, vocab 151936, K = 32, batch 1): the configuration the
-benchmark times, through the same persistent forward kernel, against the oracle.
+128, QK-norm, SwiGLU 12288, vocab 151936, K = 32): the configuration the benchmark
+times, against the oracle, with the task's bounds.
 
-A 16-token seeded prompt keeps the oracle to seconds per forward. Checked:
-- the prefill's first token, by the margin rule;
-- every draft-view and verify-view logit of one step: relative L2 <= 5e-2 and max-abs
-  <= 0.3. The GPU rounds every GEMM operand to bf16 (about six rounding points per
-  layer, relative error up to 2^-9 each) and the oracle works in float64. Over 36
-  layers of random weights these errors add like a random walk:
-  sqrt(6 * 36) * 2^-9 / sqrt(3) is about 1.7% relative, which the GPU measures (1.7% and
-  2.6%). The largest of 4.9 million logit errors sits near 5 standard deviations of
-  that, 0.1-0.2 for logits of unit scale. The 5e-2 max-abs bound of the Tiny tests
-  does not hold at this depth; the bounds here are about 2x the measured values;
-- draft and AR tokens, bit-exact where the oracle's top-2 margin > 0.1, else within
-  0.1 of its maximum;
-- accept length, committed ids and the cache length, bit-exact;
-- a second step through orthrus_decode_step (verify view with the consensus fused into
-  its last CTA): accept length, committed ids, pending token and cache length. Its
-  drafts are planted and differ from the oracle's greedy tokens, so a = 0 and the
-  committed token is the AR token, which is checked against the oracle's verify logits.
+A seeded 512-token prompt fills the cache; three consecutive decode steps follow on
+  - the persistent forward kernel (batch 1: 32 draft rows, 33 verify rows), and
+  - the per-op kernels (batch 4: 128 draft rows and 132 verify rows are more than the
+    persistent kernel takes); sequence 0 has the same prompt and is checked, the
+    other three have their own prompts.
+Checked at every step:
+  - every draft-view and verify-view logit within max-abs 5e-2 of the oracle's;
+  - draft and AR tokens bit-exact where the oracle's top-2 margin > 0.1, else within
+    0.1 of its maximum (and the oracle follows the GPU's token);
+  - accept length, committed ids, pending token and cache length bit-exact.
+
+The GPU meets the logits bound at this depth because no activation is rounded to bf16
+on its way into a tensor-core product: projections read activations as hi/lo bf16
+planes, attention reads fp16 q, softmax weights, K and V (bf16 values). With bf16
+operands throughout, 36 layers of random weights gave max-abs 0.11 (draft) and 0.2
+(verify).
 """
+import copy
+
 import numpy as np
 import pytest
 import torch
 
 import synth
-from oracle import Oracle, top2_margin
+from oracle import Oracle, accept_length, argmax_checked, top2_margin
 
 pytestmark = pytest.mark.gpu
 
 MARGIN = 0.1
-REL_L2_TOL = 5e-2   # see the module docstring for the derivation
-MAX_ABS_TOL = 0.3
+MAX_ABS_TOL = 5e-2
+K, P, STEPS = 32, 512, 3
+CAP = P + (STEPS + 1) * (K + 1) + 8
 
 
-def check_logits(gpu, ref):
-    ref = ref.numpy()
-    rel = np.linalg.norm(gpu - ref) / np.linalg.norm(ref)
-    err = float(np.abs(gpu - ref).max())
-    print(f"rel-L2 {rel:.3e} max-abs {err:.4f}")
-    assert rel <= REL_L2_TOL, rel
-    assert err <= MAX_ABS_TOL, err
-
-
-def check_tokens(gpu_ids, ref_logits):
-    for j, tok in enumerate(gpu_ids):
-        row = ref_logits[j]
-        best = int(torch.argmax(row))
-        if top2_margin(row) > MARGIN:
-            assert tok == best, (j, tok, best)
-        else:
-            assert float(row[tok]) >= float(row[best]) - MARGIN, (j, tok, best)
-
-
-def test_qwen3_8b_shape_one_step_matches_oracle():
-    from shared_kv_draft_b200 import orthrus
+@pytest.fixture(scope="module")
+def qwen(qwen_host_weights, qwen_device_weights):
     shape = synth.QWEN3_8B
-    K, P, cap = 32, 16, 128
-    w = synth.make_weights(shape, 11, 12)
-    dev = orthrus.DeviceModel(shape, w, batch=1, capacity=cap, max_block=K, max_rows=64)
+    w = qwen_host_weights
     prompt = synth.make_prompt(shape, P, 13)
-    o = Oracle(shape, w, capacity=cap)
+    o = Oracle(shape, w, capacity=CAP)
     st = o.new_state()
+    last = o.forward(st, prompt, "verify", last_only=True)  # writes the prompt's K/V
+    st.n = P
+    st.y = argmax_checked(last[0])
+    st.out = [st.y]
+    return shape, o, st, last, qwen_device_weights
 
+
+def check_logits(gpu, ref, what):
+    ref = ref.numpy()
+    err = float(np.abs(gpu - ref).max())
+    rel = float(np.linalg.norm(gpu - ref) / np.linalg.norm(ref))
+    print(f"  {what}: max-abs {err:.4f} rel-L2 {rel:.2e}")
+    assert err <= MAX_ABS_TOL, (what, err)
+
+
+def follow(tok, row):
+    """Margin rule; returns (token the oracle adopts, ambiguous?)."""
+    best = int(torch.argmax(row))
+    if top2_margin(row) > MARGIN:
+        assert tok == best, (tok, best)
+        return tok, False
+    assert float(row[tok]) >= float(row[best]) - MARGIN, (tok, best)
+    return tok, True
+
+
+def run_steps(qwen, batch):
+    from shared_kv_draft_b200 import orthrus
+    shape, o, st0, last, dev_w = qwen
+    dev = orthrus.DeviceModel(shape, dev_w, batch=batch, capacity=CAP, max_block=K, max_rows=max(64, batch * (K + 1)))
+    prompts = np.stack([synth.make_prompt(shape, P, 13 if b == 0 else 500 + b) for b in range(batch)]).astype(np.int32)
     z = lambda *s: torch.zeros(s, dtype=torch.int32, device="cuda")
-    pending = z(1)
-    dev.prefill(torch.from_numpy(prompt.astype(np.int32)).view(1, P).cuda(), [P], pending)
+    pending, draft, ar, acc, com = z(batch), z(batch, K), z(batch, K + 1), z(batch), z(batch, K + 1)
+    dlog = torch.zeros((batch, K, shape.vocab), device="cuda")
+    vlog = torch.zeros((batch, K + 1, shape.vocab), device="cuda")
+    dev.prefill(torch.from_numpy(prompts).cuda(), [P] * batch, pending)
     torch.cuda.synchronize()
-    ref_last = o.forward(o.new_state(), prompt, "verify", last_only=True)
-    y = int(pending.item())
-    check_tokens([y], ref_last)
-    o.prefill(st, prompt)
-    st.y = y
-    st.out = [y]
+    assert dev.read_status() == 0
+    st = copy.deepcopy(st0)
+    y, amb = follow(int(pending[0].item()), last[0])
+    st.y, st.out = y, [y]
+    n_amb = int(amb)
+    for step in range(STEPS):
+        dev.draft_block(pending, K, draft, dlog)
+        dev.verify_block(pending, draft, K, ar, vlog)
+        dev.accept_commit(pending, draft, ar, K, acc, com)
+        torch.cuda.synchronize()
+        assert dev.read_status() == 0
+        print(f"batch {batch} step {step} (cache {st.n}):")
+        drafts = draft[0].cpu().tolist()
+        _, dl = o.draft_block(st, K)
+        check_logits(dlog[0].cpu().numpy(), dl, "draft logits")
+        for i, t in enumerate(drafts):
+            n_amb += int(follow(t, dl[i])[1])
+        g_ref, vl = o.verify_block(st, drafts)
+        check_logits(vlog[0].cpu().numpy(), vl, "verify logits")
+        g = []
+        for j, t in enumerate(ar[0].cpu().tolist()):
+            t2, amb = follow(t, vl[j])
+            n_amb += int(amb)
+            g.append(t2)
+        a_ref, toks = o.accept_commit(st, drafts, g)
+        assert accept_length(drafts, g) == a_ref == int(acc[0].item())
+        c = com[0].cpu().tolist()
+        assert c[:a_ref + 1] == toks and all(x == -1 for x in c[a_ref + 1:])
+        assert int(dev.lens[0].item()) == st.n
+        assert int(pending[0].item()) == st.y
+        # the other sequences: consensus consistent with their own drafts and AR argmaxes
+        for b in range(1, batch):
+            d_b, g_b = draft[b].cpu().tolist(), ar[b].cpu().tolist()
+            a_b = accept_length(d_b, g_b)
+            assert int(acc[b].item()) == a_b
+            assert com[b].cpu().tolist()[:a_b + 1] == d_b[:a_b] + [g_b[a_b]]
+    print(f"batch {batch}: {n_amb} tokens within the 0.1 margin")
+    return dev, st, pending
 
-    # step 1: separate draft / verify / accept calls, with logits
-    draft, ar = z(1, K), z(1, K + 1)
-    dlog = torch.zeros((1, K, shape.vocab), device="cuda")
-    vlog = torch.zeros((1, K + 1, shape.vocab), device="cuda")
-    dev.draft_block(pending, K, draft, dlog)
-    dev.verify_block(pending, draft, K, ar, vlog)
+
+def test_qwen3_8b_persistent_kernel_three_steps(qwen):
+    """Then one more step through orthrus_decode_step (the consensus fused into the verify
+    launch) with planted drafts that cannot all match: a = 0, and the committed token is
+    the AR token, checked against the oracle's verify logits."""
+    dev, st, pending = run_steps(qwen, 1)
+    o = qwen[1]
+    z = lambda *s: torch.zeros(s, dtype=torch.int32, device="cuda")
+    tok = 7
+    g, vl = o.verify_block(st, [tok] * K)
+    if g[0] == tok:
+        tok = 8
+        g, vl = o.verify_block(st, [tok] * K)
     acc, com = z(1), z(1, K + 1)
-    dev.accept_commit(pending, draft, ar, K, acc, com)
-    torch.cuda.synchronize()
-    assert dev.read_status() == 0
-    drafts = draft[0].cpu().tolist()
-    _, dl_ref = o.draft_block(st, K)
-    check_logits(dlog[0].cpu().numpy(), dl_ref)
-    check_tokens(drafts, dl_ref)
-    _, vl_ref = o.verify_block(st, drafts)
-    check_logits(vlog[0].cpu().numpy(), vl_ref)
-    g = ar[0].cpu().tolist()
-    check_tokens(g, vl_ref)
-    a_ref, toks = o.accept_commit(st, drafts, g)
-    a = int(acc.item())
-    assert a == a_ref
-    assert com[0].cpu().tolist()[:a + 1] == toks
-    assert int(dev.lens[0].item()) == st.n == P + a + 1
-    assert int(pending.item()) == st.y
-
-    # step 2: orthrus_decode_step with planted drafts that cannot all match
-    planted = torch.full((1, K), 7, dtype=torch.int32, device="cuda")
-    _, vl2 = o.verify_block(st, [7] * K)
-    g0 = int(torch.argmax(vl2[0]))
-    if g0 == 7:  # keep a = 0 well defined: plant a token that differs from the AR argmax
-        planted.fill_(8)
-        _, vl2 = o.verify_block(st, [8] * K)
-        g0 = int(torch.argmax(vl2[0]))
-    acc2, com2 = z(1), z(1, K + 1)
     n_before = int(dev.lens[0].item())
-    dev.decode_step(pending, K, planted, acc2, com2)
+    dev.decode_step(pending, K, torch.full((1, K), tok, dtype=torch.int32, device="cuda"), acc, com)
     torch.cuda.synchronize()
     assert dev.read_status() == 0
-    assert int(acc2.item()) == 0
-    c = com2[0].cpu().tolist()
-    check_tokens([c[0]], vl2[:1])
+    assert int(acc.item()) == 0
+    c = com[0].cpu().tolist()
+    follow(c[0], vl[0])
     assert all(x == -1 for x in c[1:])
     assert int(pending.item()) == c[0]
     assert int(dev.lens[0].item()) == n_before + 1
+
+
+def test_qwen3_8b_per_op_kernels_three_steps(qwen):
+    run_steps(qwen, 4)
