@@ -727,6 +727,32 @@ __device__ __forceinline__ void fwd_epilogue(const FwdArgs& a, const QkvCtx& qc,
 
 namespace orthrus {
 
+// Accumulator columns [col, col + 32) (or + 4) of a projection. With two activation planes the
+// MMA's N covers the Mt hi rows and then the Mt lo rows of the operand, so the lo products of
+// token column j sit lo_off = Mt columns further on; they are added here (lo_off = 0: one plane).
+__device__ __forceinline__ void acc_ld32(uint32_t taddr, int col, int lo_off, float* v) {
+  tmem_ld32(taddr + col, v);
+  if (lo_off) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float w[16];
+      tmem_ld16(taddr + lo_off + col + 16 * h, w);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[16 * h + j] += w[j];
+    }
+  }
+}
+
+__device__ __forceinline__ void acc_ld4(uint32_t taddr, int col, int lo_off, float* v) {
+  tmem_ld4(taddr + col, v);
+  if (lo_off) {
+    float w[4];
+    tmem_ld4(taddr + lo_off + col, w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] += w[j];
+  }
+}
+
 // Greedy consensus (verify launch) and counter reset; run by the last CTA to
 // finish, when every other CTA has left the kernel.
 __device__ inline void fwd_finalize(const FwdArgs& a, int n_ph) {
@@ -1074,7 +1100,8 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         const int buf = seg & 1, use = seg >> 1;
         ++seg;
         const int nt = t;
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * 128;
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * 256;
+        const int lo_off = gp.planes == 2 ? a.Mt : 0;
         const bool whole = seg_start == (long long)t * kc && seg_end == (long long)(t + 1) * kc;
         float v[32];
         if (whole) {
@@ -1086,9 +1113,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           tc_fence_after();
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
             if (m0 == 32 && n2 > 0) break;  // rows 32.. went with the first call
-            tmem_ld32(taddr + m0, v);
+            acc_ld32(taddr, m0, lo_off, v);
             float v2[4];
-            if (m0 == 0 && n2 > 0) tmem_ld4(taddr + 32, v2);
+            if (m0 == 0 && n2 > 0) acc_ld4(taddr, 32, lo_off, v2);
             fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, m0 == 0 && n2 > 0 ? v2 : nullptr, row, m0, nt, m_valid,
                                  epi, red, rstd_s, gam_tile(nt));
           }
@@ -1120,7 +1147,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           const int slot = 2 * c + (t == first_tile ? 0 : 1);
           float4* part = reinterpret_cast<float4*>(a.partial + (size_t)slot * (128 * 128)) + row;
           for (int m0 = 0; m0 < a.Mt; m0 += 32) {
-            tmem_ld32(taddr + m0, v);
+            acc_ld32(taddr, m0, lo_off, v);
             if (add_h) {
               float hv[32];
 #pragma unroll
@@ -1187,9 +1214,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
           if (m0 == 32 && n2 > 0) break;  // rows 32.. went with the first call
           const bool fuse = m0 == 0 && n2 > 0;
-          tmem_ld32(taddr + m0, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
+          acc_ld32(taddr, m0, lo_off, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
           float v2[4];
-          if (fuse) tmem_ld4(taddr + 32, v2);
+          if (fuse) acc_ld4(taddr, 32, lo_off, v2);
           int cc = c_lo + 1;
           if (m0 == 0) {
             add2(v, x);
@@ -1575,6 +1602,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   tc_fence_after();
   const FwdGeom g = *geom_s;
   const uint32_t tmem_base = *tmem_slot;
+  // TMEM: two projection accumulators of up to 256 columns (2 Mt: hi and lo products) at 0 and 256.
+  // The attention tiles alias the second one: a projection accumulator is read by its epilogue
+  // before the phase completes, and attention MMAs wait for the q/k/v phase's completion (the Q
+  // tile); the next projection's MMAs wait for the attention phase's output (their activations).
   const uint32_t tS = tmem_base + 256;  // attention scores: 64 columns
   const uint32_t tO = tmem_base + 320;  // attention P V tile: d columns
 
@@ -1643,9 +1674,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 break;
               }
               if (u == u0) tl_mark<TL>(a, n_ph, p, TL_X0);
-              // box [plane][k chunk][Mt rows][64]
+              // box [k chunk][plane][Mt rows][64] (one plane for the LM head)
               mbar_arrive_expect_tx(&full[s], (uint32_t)a.Mt * 256u * (uint32_t)gp.planes);
-              if (gp.planes == 2) tma_load_4d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k, 0);
+              if (gp.planes == 2) tma_load_4d(st + 32768, gp.mx, &full[s], 0, 0, 0, 2 * k);
               else tma_load_3d(st + 32768, gp.mx, &full[s], 0, 0, 2 * k);
             }
             last_ph[s] = (int)ph;
@@ -1728,7 +1759,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
-      const uint32_t idesc_g = idesc_bf16(128, a.Mt, false);
+      const uint32_t idesc_g = idesc_bf16(128, a.Mt, false);       // one activation plane (LM head)
+      const uint32_t idesc_g2 = idesc_bf16(128, 2 * a.Mt, false);  // hi rows then lo rows
       const uint32_t idS = idesc_f16(128, 64, false);  // fp16 q and K
       const uint32_t idO = idesc_f16(128, d, true);    // fp16 P and V
       const uint32_t pa = smem_u32(scr);
@@ -1755,7 +1787,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + buf * 128;
+            const uint32_t d_tmem = tmem_base + buf * 256;
             for (; u < seg_end; ++u, ++it) {
               const int s = it % S;
               const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -1769,17 +1801,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               tc_fence_after();
               const uint32_t wa = smem_u32(stage_ptr(s));
               const uint32_t xa = wa + 32768;
-              const uint32_t x_lo = 2u * (uint32_t)a.Mt * 128u;  // lo plane after the hi plane's two chunks
+              // activation box [k chunk][plane][Mt][64]: per chunk, the B operand is the Mt hi rows
+              // followed by the Mt lo rows, one MMA of N = 2 Mt (the weights are read once)
+              const uint32_t x_chunk = (uint32_t)gp.planes * (uint32_t)a.Mt * 128u;
+              const uint32_t idx = gp.planes == 2 ? idesc_g2 : idesc_g;
+              // a descriptor's start address is (address >> 4) in its low 14 bits: an offset into
+              // shared memory (below 256 KB) is added there directly
+              const uint64_t wd0 = sw128_desc(wa, 16, 1024), xd0 = sw128_desc(xa, 16, 1024);
 #pragma unroll
               for (int c2 = 0; c2 < 2; ++c2) {  // the two 64-wide k chunks of the unit
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t wd = sw128_desc(wa + c2 * 16384 + kk * 32, 16, 1024);
-                  const uint32_t xo = c2 * (uint32_t)a.Mt * 128u + kk * 32;
-                  mma_ss(d_tmem, wd, sw128_desc(xa + xo, 16, 1024), idesc_g,
-                              (u > seg_start || c2 > 0 || kk > 0) ? 1u : 0u);
-                  if (gp.planes == 2) mma_ss(d_tmem, wd, sw128_desc(xa + x_lo + xo, 16, 1024), idesc_g, 1u);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_ss(d_tmem, wd0 + (uint64_t)((c2 * 16384 + kk * 32) >> 4),
+                         xd0 + (uint64_t)((c2 * x_chunk + kk * 32) >> 4), idx,
+                         (u > seg_start || c2 > 0 || kk > 0) ? 1u : 0u);
               }
               mma_commit(&empty[s]);
             }

@@ -51,7 +51,7 @@ struct QkvEpi {
 
 struct GemmArgs {
   int N, Kd, M;              // weight rows, reduction length, valid token rows
-  int Mt, mt_alloc;          // token tile (multiple of 16, <= 128), TMEM columns per accumulator
+  int Mt, mt_alloc;          // token tile (multiple of 16, <= 128), TMEM columns per accumulator (>= planes Mt)
   int m_tiles, n_tiles, k_chunks;
   long long total_units;
   int stages;
@@ -323,7 +323,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, a.Mt, false);
+      // with two planes the B operand is the Mt hi rows then the Mt lo rows: one MMA of N = 2 Mt
+      const uint32_t idesc = idesc_bf16(128, a.planes * a.Mt, false);
       int it = 0, seg = 0;
       long long u = u0;
       bool ok = true;
@@ -343,13 +344,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t wa = smem_u32(smem + (size_t)s * stage_bytes);
           const uint32_t xa = wa + 16384;
-          const uint32_t x_lo = (uint32_t)a.Mt * 128u;
+          // 32-byte k steps: (32 >> 4) added to the descriptors' start-address field
+          const uint64_t wd0 = sw128_desc(wa, 16, 1024), xd0 = sw128_desc(xa, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t wd = sw128_desc(wa + kk * 32, 16, 1024);
-            mma_ss(d_tmem, wd, sw128_desc(xa + kk * 32, 16, 1024), idesc, (u > seg_start || kk > 0) ? 1u : 0u);
-            if (a.planes == 2) mma_ss(d_tmem, wd, sw128_desc(xa + x_lo + kk * 32, 16, 1024), idesc, 1u);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(d_tmem, wd0 + (uint64_t)(2 * kk), xd0 + (uint64_t)(2 * kk), idesc, (u > seg_start || kk > 0) ? 1u : 0u);
           mma_commit(&empty[s]);
         }
         if (!ok) break;
@@ -364,6 +363,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     griddep_wait();  // outputs and shared scratch are touched only after the predecessor finished
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
+    // accumulator columns [col, col + 32); with two planes the lo products sit Mt columns on
+    auto acc_ld = [&](uint32_t taddr, int col, float* v) {
+      tmem_ld32(taddr + col, v);
+      if (a.planes == 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float w[16];
+          tmem_ld16(taddr + a.Mt + col + 16 * h, w);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * h + j] += w[j];
+        }
+      }
+    };
     int seg = 0;
     long long u = u0;
     const int first_tile = (int)(u0 / kc);
@@ -387,7 +399,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!got) break;
       if (whole) {
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
-          tmem_ld32(taddr + m0, v);
+          acc_ld(taddr, m0, v);
           epilogue_group<EPI>(a, v, row, m0, mt, nt, m_valid, epi, red);
         }
         tc_fence_before();
@@ -399,7 +411,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int slot = 2 * c + (t == first_tile ? 0 : 1);
         float* part = a.partial + (size_t)slot * (128 * 128) + (size_t)row * a.Mt;
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
-          tmem_ld32(taddr + m0, v);
+          acc_ld(taddr, m0, v);
           const int n4 = min(32, a.Mt - m0) / 4;
 #pragma unroll
           for (int q = 0; q < 8; ++q)

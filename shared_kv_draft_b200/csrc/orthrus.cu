@@ -110,11 +110,12 @@ bool map_planes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, 
   return map_nd(m, base, 3, dims, strides, box);
 }
 
-// The same as (64 columns, rows, cols/64 chunks, plane): a box of (64, box_rows, 2, 2) is two
-// consecutive 64-wide k chunks of both planes, laid out [plane][chunk][row][64].
+// The same as (64 columns, rows, plane, cols/64 chunks): a box of (64, box_rows, 2, 2) is two
+// consecutive 64-wide k chunks of both planes, laid out [chunk][plane][row][64], so that per
+// chunk the hi rows and then the lo rows form one MMA operand of 2 box_rows rows.
 bool map_kpair_planes(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
-  const uint64_t dims[4] = {64, rows, cols / 64, 2};
-  const uint64_t strides[3] = {cols * 2, 128, cols * rows * 2};
+  const uint64_t dims[4] = {64, rows, 2, cols / 64};
+  const uint64_t strides[3] = {cols * 2, cols * rows * 2, 128};
   const uint32_t box[4] = {64, box_rows, 2, 2};
   return map_nd(m, base, 4, dims, strides, box);
 }
@@ -380,12 +381,12 @@ cudaError_t launch_gemm(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs
   a.M = M;
   a.m_tiles = (M + 127) / 128;
   a.Mt = a.m_tiles > 1 ? 128 : round_up(std::max(M, 1), 16);
-  a.mt_alloc = std::max(32, next_pow2(a.Mt));
+  a.planes = std::max(1, a.planes);
+  a.mt_alloc = std::max(32, next_pow2(a.planes * a.Mt));  // hi and lo products side by side
   a.n_tiles = (EPI == EPI_SWIGLU) ? N / 128 : N / 128;  // SwiGLU: N = 2F, a tile = 64 gate + 64 up rows
   a.k_chunks = Kd / 64;
   a.total_units = (long long)a.m_tiles * a.n_tiles * a.k_chunks;
   const int G = (int)std::min<long long>(num_sms(), a.total_units);
-  a.planes = std::max(1, a.planes);
   const size_t fixed = gemm_smem_bytes(a.Mt, 0, a.planes);
   const size_t stage = 16384 + (size_t)a.Mt * 128 * a.planes;
   a.stages = (int)std::min<size_t>(12, (kSmemLimit - fixed) / stage);
