@@ -1173,8 +1173,9 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         // Head owner. The other contributors stored their parts at the start of their
         // ranges, long before this CTA's own part (the end of its range) is accumulated:
-        // their count is awaited and their first token group loaded while the MMAs of
-        // the last k units still run.
+        // their count is awaited and the first token group of all of them summed, in k
+        // order, while the MMAs of the last k units still run; only the add of that sum
+        // to the own part is left for when the accumulator is ready.
         int n_contrib = 0;
         for (int cc = c_lo; cc <= c_hi; ++cc) n_contrib += ust_s[cc + 1] > ust_s[cc];
         bool ready = false;
@@ -1189,21 +1190,36 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           ok = false;
           break;
         }
-        int cc0 = c_lo + 1, s0, s1;
-        gather2(cc0, c_hi, s0, s1, t);
-        const int f0 = s0, f1 = s1;  // the first round's slots (s0, s1 move on in later rounds)
-        float4 x[2][8];
-        load2(x, s0, s1, 0);
-        // a second token group (the 33rd row of a K = 32 verify block) is usually one float4
-        // row: the same contributors' row 8 is loaded now too
-        float4 x2[2];
+        // pre = c_lo+1 + c_lo+2 + ... + c_hi (token rows 0..31, and the second group's rows
+        // 32..35 when they ride with the first call); the own part is added to it last
+        float pre[32], pre2[4];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int sl = q == 0 ? s0 : s1;
-          x2[q] = (sl >= 0 && m_valid > 32)
-                      ? ld_f4_hint(reinterpret_cast<const float4*>(a.partial + (size_t)sl * (128 * 128)) + 8 * 128 + row,
-                                   pol_drop)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 32; ++j) pre[j] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pre2[k] = 0.f;
+        for (int cc = c_lo + 1; cc <= c_hi;) {
+          int s0, s1;
+          gather2(cc, c_hi, s0, s1, t);
+          float4 x[2][8];
+          load2(x, s0, s1, 0);
+          float4 x2[2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int sl = q == 0 ? s0 : s1;
+            x2[q] = (sl >= 0 && n2 > 0)
+                        ? ld_f4_hint(reinterpret_cast<const float4*>(a.partial + (size_t)sl * (128 * 128)) + 8 * 128 +
+                                         row,
+                                     pol_drop)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          add2(pre, x);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            pre2[0] += x2[q].x;
+            pre2[1] += x2[q].y;
+            pre2[2] += x2[q].z;
+            pre2[3] += x2[q].w;
+          }
         }
         if (!bar_wait_all(&accf[buf], (uint32_t)use & 1u, 13)) {
           ok = false;
@@ -1214,63 +1230,31 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         for (int m0 = 0; m0 < a.Mt; m0 += 32) {
           if (m0 == 32 && n2 > 0) break;  // rows 32.. went with the first call
           const bool fuse = m0 == 0 && n2 > 0;
-          acc_ld32(taddr, m0, lo_off, v);  // own part first: the k order is c_lo, c_lo+1, ..., c_hi
+          acc_ld32(taddr, m0, lo_off, v);  // own part: the first k units of the tile
           float v2[4];
           if (fuse) acc_ld4(taddr, 32, lo_off, v2);
-          int cc = c_lo + 1;
           if (m0 == 0) {
-            add2(v, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += pre[j];
             if (fuse) {
 #pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                v2[0] += x2[q].x;
-                v2[1] += x2[q].y;
-                v2[2] += x2[q].z;
-                v2[3] += x2[q].w;
-              }
+              for (int k = 0; k < 4; ++k) v2[k] += pre2[k];
             }
-            cc = cc0;
-          } else if (m0 == 32) {
-            // the first round's contributors: row 8 prefetched, rows 9.. (tokens 36..) loaded here
+          } else {
+            // further token groups (blocks of more than 36 rows): the contributors in the same
+            // k order, summed first as for the first group, then added to the own part
+            float sum[32];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int sl = q == 0 ? f0 : f1;
-              const float4* pp = reinterpret_cast<const float4*>(a.partial + (size_t)(sl < 0 ? 0 : sl) * (128 * 128)) +
-                                 8 * 128 + row;
-              v[0] += x2[q].x;
-              v[1] += x2[q].y;
-              v[2] += x2[q].z;
-              v[3] += x2[q].w;
-#pragma unroll
-              for (int q4 = 1; q4 < 8; ++q4)
-                if (sl >= 0 && 32 + 4 * q4 < m_valid) {
-                  const float4 y = ld_f4_hint(pp + (size_t)q4 * 128, pol_drop);
-                  v[4 * q4] += y.x;
-                  v[4 * q4 + 1] += y.y;
-                  v[4 * q4 + 2] += y.z;
-                  v[4 * q4 + 3] += y.w;
-                }
+            for (int j = 0; j < 32; ++j) sum[j] = 0.f;
+            for (int cc = c_lo + 1; cc <= c_hi;) {
+              int s0, s1;
+              gather2(cc, c_hi, s0, s1, t);
+              float4 x[2][8];
+              load2(x, s0, s1, m0);
+              add2(sum, x);
             }
-            cc = cc0;
-          }
-          while (cc <= c_hi) {
-            gather2(cc, c_hi, s0, s1, t);
-            load2(x, s0, s1, m0);
-            if (fuse) {
 #pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int sl = q == 0 ? s0 : s1;
-                if (sl >= 0) {
-                  const float4 y = ld_f4_hint(
-                      reinterpret_cast<const float4*>(a.partial + (size_t)sl * (128 * 128)) + 8 * 128 + row, pol_drop);
-                  v2[0] += y.x;
-                  v2[1] += y.y;
-                  v2[2] += y.z;
-                  v2[3] += y.w;
-                }
-              }
-            }
-            add2(v, x);
+            for (int j = 0; j < 32; ++j) v[j] += sum[j];
           }
           if (et == 0) tl_mark<TL>(a, n_ph, p, TL_S_LOAD);
           fwd_epilogue<D_HEAD>(a, qc, lens_s, gp.epi, v, fuse ? v2 : nullptr, row, m0, nt, m_valid, epi, red, rstd_s,
