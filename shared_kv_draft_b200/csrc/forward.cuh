@@ -1295,10 +1295,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         // the next P V. O is read into registers once, after the last tile.
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; j < t.tiles; ++j, it += 2, ++ta) {
-          if (!bar_wait_all(s_full, (uint32_t)ta & 1u, 14)) {
+          // score buffer ta & 1; its barrier completes once per use, every second tile
+          if (!bar_wait_all(&s_full[(ta & 1) * 3], (uint32_t)(ta >> 1) & 1u, 14)) {
             ok = false;
             break;
           }
+          const uint32_t tSb = (ta & 1) ? tS + 192 : tS;  // the second buffer sits at column 448
           if (et == 0) tl_mark<TL>(a, n_ph, p, j == 0 ? TL_R0 : TL_S_ACC);  // score tile ready
           tc_fence_after();
           const int key0 = t.key_lo + j * 64;
@@ -1311,7 +1313,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 32) {
-            tmem_ld32(tS + lane_base + c0, sv);
+            tmem_ld32(tSb + lane_base + c0, sv);
 #pragma unroll
             for (int tt = 0; tt < 32; tt += 4) {
               mx0 = fmaxf(mx0, c0 + tt < nv ? sv[tt] : -INFINITY);
@@ -1345,7 +1347,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 32) {
-            tmem_ld32(tS + lane_base + c0, sv);
+            tmem_ld32(tSb + lane_base + c0, sv);
             uint32_t pk[16];
 #pragma unroll
             for (int tt = 0; tt < 32; tt += 2) {
@@ -1525,7 +1527,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   uint64_t* empty = bars + kMaxStages;
   uint64_t* accf = bars + 2 * kMaxStages;  // [2]
   uint64_t* acce = accf + 2;               // [2]
-  uint64_t* s_full = acce + 2;
+  uint64_t* s_full = acce + 2;  // [0] and [3]: scores of even / odd key tiles ready
   uint64_t* p_full = s_full + 1;
   uint64_t* o_full = s_full + 2;
   uint64_t* done = s_full + 4;
@@ -1551,6 +1553,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
       mbar_init(&acce[b], 4);
     }
     mbar_init(s_full, 1);
+    mbar_init(s_full + 3, 1);  // second score buffer
     mbar_init(p_full, 4);
     mbar_init(o_full, 1);
     mbar_init(done, 1);
@@ -1590,8 +1593,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   // The attention tiles alias the second one: a projection accumulator is read by its epilogue
   // before the phase completes, and attention MMAs wait for the q/k/v phase's completion (the Q
   // tile); the next projection's MMAs wait for the attention phase's output (their activations).
-  const uint32_t tS = tmem_base + 256;  // attention scores: 64 columns
-  const uint32_t tO = tmem_base + 320;  // attention P V tile: d columns
+  const uint32_t tS = tmem_base + 256;   // attention scores: 64 columns (even key tiles)
+  const uint32_t tO = tmem_base + 320;   // attention P V tile: d columns
+  const uint32_t tS2 = tmem_base + 448;  // scores of odd key tiles
 
   if (warp == 0 || warp == 6) {
     // ============ TMA producers: warp 0 streams weight tiles, warp 6 activations ============
@@ -1817,23 +1821,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               ok = false;
               break;
             }
+            // S = Q K^T of key tile jj (ring item itj, tile counter taj) into score buffer taj & 1
+            auto issue_s = [&](int jj, int itj, int taj) -> bool {
+              const int ks = itj % S;
+              const int rr = mbar_wait_code(&full[ks], (uint32_t)(itj / S) & 1u, a.status);
+              if (rr != 1) {
+                fwd_diag(a, rr, 8, p, itj, ks);
+                return false;
+              }
+              tc_fence_after();
+              const uint64_t qd0 = sw128_desc(qa, 16, 1024), kd0 = sw128_desc(smem_u32(stage_ptr(ks)), 16, 1024);
+              const uint32_t ts = (taj & 1) ? tS2 : tS;
+#pragma unroll
+              for (int kk = 0; kk < d / 16; ++kk)
+                mma_ss(ts, qd0 + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                       kd0 + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
+              mma_commit(&s_full[(taj & 1) * 3]);
+              mma_commit(&empty[ks]);
+              if (jj == t.tiles - 1) mma_commit(q_empty);  // last read of this unit's Q tile
+              return true;
+            };
+            if (!issue_s(0, it, ta)) {
+              ok = false;
+              break;
+            }
             for (int j = 0; ok && j < t.tiles; ++j, it += 2, ++ta) {
-              const int ks = it % S, vs = (it + 1) % S;
-              r = mbar_wait_code(&full[ks], (uint32_t)(it / S) & 1u, a.status);
-              if (r != 1) {
-                fwd_diag(a, r, 8, p, it, ks);
+              const int vs = (it + 1) % S;
+              // the next tile's scores go into the other buffer while the softmax warps work on
+              // this one (its previous contents, tile j - 1, were read before P of j - 1)
+              if (j + 1 < t.tiles && !issue_s(j + 1, it + 2, ta + 1)) {
                 ok = false;
                 break;
               }
-              tc_fence_after();
-              const uint32_t ka = smem_u32(stage_ptr(ks));
-#pragma unroll
-              for (int kk = 0; kk < d / 16; ++kk)
-                mma_ss(tS, sw128_desc(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                            sw128_desc(ka + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
-              mma_commit(s_full);
-              mma_commit(&empty[ks]);
-              if (j == t.tiles - 1) mma_commit(q_empty);  // last read of this unit's Q tile
               // P of this tile written (and O rescaled) by the softmax warps, V landed
               r = mbar_wait_code(p_full, (uint32_t)ta & 1u, a.status);
               if (r == 1) {

@@ -818,8 +818,17 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->ss = (float*)(base + wl.ss);
   P->ss_ld = wl.ss_ld;
   P->mega_slots = wl.mega_slots;
-  // attention chunk of the persistent kernel: at most kMaxChunks - 2 chunks over the whole capacity
+  // attention chunk of the persistent kernel, fixed per plan (so verify rows and plain AR rows
+  // see the same chunk boundaries): at most kMaxChunks - 2 chunks over the whole capacity, and
+  // long enough that a full cache's verify-view units (sequence, KV head, row tile, chunk) fit
+  // one wave of CTAs
   P->fwd_ck = std::max(64, round_up((P->cap + kMaxChunks - 3) / (kMaxChunks - 2), 64));
+  {
+    const int G = cfg->n_heads / cfg->n_kv_heads;
+    const int slots_v = P->B * cfg->n_kv_heads * ((G * (max_block + 1) + 127) / 128);
+    const int sms = num_sms();
+    P->fwd_ck = std::max(P->fwd_ck, round_up((int)(((long long)P->cap * slots_v + sms - 1) / sms), 64));
+  }
   P->fwd_att_o = (float*)(base + wl.fwd_att_o);
   P->fwd_att_ml = (float2*)(base + wl.fwd_att_ml);
   P->norms_off = norms_off;
