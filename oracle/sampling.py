@@ -22,7 +22,9 @@ Sampling", 2023), applied to the Orthrus block:
   rejection; a = number accepted;
 * the last committed token is drawn with a further uniform v: from the
   residual max(0, p_a - q_a) (normalised) when d_{a+1} was rejected, else
-  from p_K (the bonus token);
+  from p_K (the bonus token). The pages leave open a residual that is zero
+  everywhere, which needs p_a == q_a and a draft of zero draft probability;
+  the reading here draws from p_a then, the target distribution itself;
 * committed = d_1..d_a and that token; the cache and pending-token bookkeeping
   is the greedy step's (n += a + 1, y = last committed).
 
@@ -108,7 +110,10 @@ def speculative_accept(drafts, q, p, u_accept, v_final):
             break
     if a < K:
         resid = torch.clamp(_f64(p[a]) - _f64(q[a]), min=0.0)
-        last = inverse_cdf(resid, float(v_final))
+        # The residual is empty only when p_a == q_a and d_{a+1} lies outside q_a's support
+        # (a draft the draft view gives probability zero, so never one drawn from it): the
+        # rejection then says nothing and the last token is drawn from p_a itself.
+        last = inverse_cdf(resid if float(resid.sum()) > 0 else _f64(p[a]), float(v_final))
     else:
         last = inverse_cdf(_f64(p[K]), float(v_final))
     return a, [int(t) for t in drafts[:a]] + [last]

@@ -354,3 +354,105 @@ def test_sampled_decode_matches_oracle(shape):
         assert np.array_equal(acc.cpu().numpy(), A) and np.array_equal(com.cpu().numpy(), Cm)
     assert dev.read_status() == 0
     assert [int(x) for x in dev.lens] == [st.n for st in states]
+
+
+# ---- edges of the inverse CDF and of the residual ------------------------------------------
+
+V_BELOW_ONE = np.float32(1.0 - 2.0 ** -24)  # the largest fp32 uniform below 1
+
+
+def test_sample_tokens_edges_of_the_cdf():
+    # Rows whose draw is the same index in any precision, at the top end of [0, 1): v * Z lies
+    # within 6e-8 of the total, where the kernel's fallbacks decide the token when its running
+    # sums round past the target, or reach it only at zero-weight elements.
+    V = 3149  # four CDF tiles, the last one ragged
+    rng = np.random.default_rng(91)
+    x = np.full((4, V), -np.inf, dtype=np.float32)
+    x[0, :1500] = rng.normal(-30.0, 1.0, 1500)  # tiny weights before one dominant token,
+    x[0, 1500] = 0.0                             # nothing after it
+    x[1, 0] = 3.0                                # one token, the first
+    x[2, :1000] = rng.normal(0.0, 1.0, 1000)     # the first tile only: the last positive index
+    x[3, 2048:V] = rng.normal(0.0, 1.0, V - 2048)  # the last two tiles only, v = 0: the first of them
+    u = np.array([V_BELOW_ONE, V_BELOW_ONE, V_BELOW_ONE, 0.0], dtype=np.float32)
+    out, status = i32(4), i32(1)
+    lib().sample_tokens(torch.from_numpy(x).cuda(), 1.0, torch.from_numpy(u).cuda(), out, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = [inverse_cdf(tempered_weights(torch.from_numpy(x[r]), 1.0), float(u[r])) for r in range(4)]
+    assert ref == [1500, 0, 999, 2048]
+    assert out.cpu().tolist() == ref
+
+
+def test_accept_sample_edges_of_the_residual():
+    # Three sequences, K = 2, uniforms at the top end of [0, 1):
+    #  b = 0: verify row 0 equals draft row 0 except one raised logit j, so p_0 < q_0 everywhere
+    #         but at j: d_1 is rejected (p/q = Z_d / Z_v well below u) and the residual is
+    #         positive only at j, the last token for any v;
+    #  b = 1: p_0 == q_0 exactly and d_1 outside their support: rejected, the residual is zero
+    #         everywhere, and the last token is drawn from p_0 (one-hot: its token);
+    #  b = 2: p == q exactly on rows 0 and 1 with each draft the row's top token (q = 1 after the
+    #         max shift): both accepted for u just below 1, and the bonus token drawn from p_2
+    #         with v just below 1 is its dominant token (nothing after it has weight).
+    shape = replace(synth.TINY, name="tiny_v1024", n_layers=1)
+    w = synth.make_weights(shape, 75, 76)
+    B, K, V = 3, 2, 1024
+    dev = lib().DeviceModel(shape, w, batch=B, capacity=64, max_block=K, max_rows=64)
+    rng = np.random.default_rng(92)
+    dl = rng.normal(0.0, 1.0, (B, K, V)).astype(np.float32)
+    vl = dl.copy()
+    vl = np.concatenate([vl, rng.normal(0.0, 1.0, (B, 1, V)).astype(np.float32)], axis=1)
+    drafts = np.zeros((B, K), dtype=np.int32)
+    # b = 0
+    top = int(np.argmax(dl[0, 0]))
+    j = int(np.argsort(dl[0, 0])[-3])            # third largest: stays below the max once raised
+    vl[0, 0, j] = dl[0, 0, j] + np.float32(0.9 * (dl[0, 0, top] - dl[0, 0, j]))
+    drafts[0] = [(j + 1) % V if (j + 1) % V != top else (j + 2) % V, 5]
+    # b = 1
+    dl[1, 0] = -np.inf
+    dl[1, 0, 321] = 0.5
+    vl[1, 0] = dl[1, 0]
+    drafts[1] = [100, 7]
+    # b = 2
+    for i in range(K):
+        vl[2, i] = dl[2, i]
+        drafts[2, i] = int(np.argmax(dl[2, i]))
+    vl[2, K, :] = -np.inf
+    vl[2, K, :600] = rng.normal(-30.0, 1.0, 600)
+    vl[2, K, 600] = 1.0
+    ua = np.full((B, K), V_BELOW_ONE, dtype=np.float32)
+    uf = np.full((B,), V_BELOW_ONE, dtype=np.float32)
+    pending, acc, com = i32(B), i32(B), i32(B, K + 1)
+    dev.lens.fill_(10)
+    dev.accept_sample(pending, torch.from_numpy(drafts).cuda(), torch.from_numpy(dl).cuda(),
+                      torch.from_numpy(vl).cuda(), K, 1.0, torch.from_numpy(ua).cuda(), torch.from_numpy(uf).cuda(),
+                      acc, com)
+    torch.cuda.synchronize()
+    assert dev.read_status() == 0
+    expect = [(0, [j]), (0, [321]), (2, [int(drafts[2, 0]), int(drafts[2, 1]), 600])]
+    for b in range(B):
+        a_ref, toks = accept_sample_logits([int(t) for t in drafts[b]], torch.from_numpy(dl[b]),
+                                           torch.from_numpy(vl[b]), 1.0, ua[b], uf[b])
+        assert (a_ref, toks) == expect[b], b
+        assert int(acc[b]) == a_ref
+        assert com[b].cpu().tolist() == toks + [-1] * (K + 1 - len(toks))
+        assert int(pending[b]) == toks[-1] and int(dev.lens[b]) == 10 + a_ref + 1
+
+
+def test_accept_sample_with_a_row_of_no_finite_logit_commits_nothing():
+    # A verify row whose logits are all -inf has no distribution: the status word takes
+    # ORTHRUS_ERR_NAN and no sequence commits anything.
+    shape = replace(synth.TINY, name="tiny_v1024", n_layers=1)
+    w = synth.make_weights(shape, 77, 78)
+    B, K, V = 2, 3, 1024
+    dev = lib().DeviceModel(shape, w, batch=B, capacity=64, max_block=K, max_rows=64)
+    dl = torch.zeros((B, K, V), device="cuda")
+    vl = torch.zeros((B, K + 1, V), device="cuda")
+    vl[0, K] = float("-inf")
+    pending, acc, com = i32(B), i32(B), i32(B, K + 1)
+    dev.lens.fill_(9)
+    dev.accept_sample(pending, i32(B, K), dl, vl, K, 1.0, torch.full((B, K), 0.5, device="cuda"),
+                      torch.full((B,), 0.5, device="cuda"), acc, com)
+    torch.cuda.synchronize()
+    assert dev.read_status() == lib().ERR_NAN
+    assert acc.cpu().tolist() == [-1, -1] and (com == -1).all()
+    assert dev.lens.cpu().tolist() == [9, 9]

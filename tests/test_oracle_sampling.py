@@ -303,3 +303,23 @@ def test_sampled_step_on_the_decoder_reduces_to_the_greedy_step_when_cold():
         drafts, a, toks = osamp.sampled_step(m, cold, K, 1e-4, ud[0], ua[0], float(uf[0]))
         assert drafts == d_ref and a == a_ref and toks == toks_ref
         assert cold.n == greedy.n and cold.y == greedy.y
+
+
+def test_empty_residual_draws_from_the_target():
+    # p_0 == q_0 and a draft outside q_0's support: u * q(d) = 0 is not < p(d) = 0, so the draft
+    # is rejected and max(0, p_0 - q_0) is zero everywhere. The committed token must still be
+    # distributed as p_0 (the frozen model's sampling distribution): one-hot p_0 forces its
+    # token, a spread p_0 gives p_0's frequencies on a stratified grid of v.
+    one_hot = np.array([0.0, 0.0, 1.0, 0.0])
+    for u in (0.0, 0.5, 0.999):
+        for v in (0.0, 0.5, 0.999):
+            a, toks = speculative_accept([1], [one_hot], [one_hot, one_hot], [u], v)
+            assert a == 0 and toks == [2]
+    p0 = np.array([0.1, 0.0, 0.6, 0.3])
+    N = 1000
+    counts = np.zeros(4)
+    for i in range(N):
+        a, toks = speculative_accept([1], [p0], [p0, one_hot], [0.5], (i + 0.5) / N)
+        assert a == 0
+        counts[toks[0]] += 1
+    assert np.allclose(counts / N, p0, atol=1.5 / N)
