@@ -931,8 +931,8 @@ def main():
         "decode_step_tensor": {"achieved_tflops": round(r["flops"] / (r["ms"] * 1e-3) / 1e12, 1),
                                "peak_tflops": r["tf_peak"],
                                "frac": round(r["flops"] / (r["ms"] * 1e-3) / 1e12 / r["tf_peak"], 4),
-                               "note": "algorithmic flops; projections issue two MMAs per chunk (hi and lo "
-                                       "activation planes)"},
+                               "note": "algorithmic flops; the layer projections run on both activation planes "
+                                       "(hi and lo rows in one MMA), twice these flops on the tensor pipe"},
         "prefill": r["prefill"],
         "roofline": r["roofline"],
         "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in v.items()}
