@@ -211,6 +211,61 @@ def step_flops(shape, B, K, n_list):
     return 2.0 * params * B * (2 * K + 1) + att
 
 
+def greedy_streams(m, pending, n, dev):
+    """The next n greedy tokens of every sequence from the current device state, by K = 0 steps
+    (the verify view on the pending token, then its commit): [B][n], column 0 the pending token.
+    Advances the cache lengths and pending tokens; callers restore them."""
+    import torch
+    B = pending.numel()
+    sd = torch.zeros((n, B), dtype=torch.int32, device=dev)
+    sd[0] = pending
+    ar1 = torch.zeros((B, 1), dtype=torch.int32, device=dev)
+    acc1 = torch.zeros((B,), dtype=torch.int32, device=dev)
+    for j in range(1, n):
+        m.verify_block(pending, None, 0, ar1)
+        m.accept_commit(pending, None, ar1, 0, acc1, sd[j])
+    torch.cuda.synchronize(dev)
+    if m.read_status() != 0:
+        raise RuntimeError(f"device status {m.read_status()} while building the greedy streams")
+    return sd.cpu().numpy().T.copy()
+
+
+def planted_step(m, pending, dev, stream, jpos, a_plan, K, V, rng, acc, com):
+    """One untimed decode step on drafts planted from the greedy streams (accept lengths a_plan),
+    read back on the host. The streams come from the K = 0 path; a verify block of more than 128
+    token rows runs on the per-op kernels, whose sums run in another order, so at a near tie its
+    argmax can leave the stream. The committed tokens then replace the stream there and the rest
+    of every stream is rebuilt from the new state. Returns (drafts, accept lengths, committed ids,
+    rebuilt); jpos advances by each sequence's committed count."""
+    import torch
+    B = len(jpos)
+    d = np.stack([synth.planted_drafts(stream[b], jpos[b], int(a_plan[b]), K, V, rng)
+                  for b in range(B)]).astype(np.int32)
+    m.decode_step(pending, K, torch.from_numpy(d).to(dev), acc, com)
+    a = acc.cpu().numpy().astype(np.int64)
+    c = com.cpu().numpy()
+    if m.read_status() != 0 or np.any(a < 0):
+        raise RuntimeError(f"device status {m.read_status()} in a planted step")
+    left = False
+    for b in range(B):
+        got = c[b, :a[b] + 1]
+        if a[b] != a_plan[b] or not np.array_equal(got, stream[b, jpos[b] + 1:jpos[b] + a[b] + 2]):
+            left = True
+        stream[b, jpos[b] + 1:jpos[b] + a[b] + 2] = got
+        jpos[b] += int(a[b]) + 1
+    if left:
+        lens0, pend0 = m.lens.clone(), pending.clone()
+        # as many tokens as the longest cache has room for (a later rebuild extends the rest)
+        n = min(stream.shape[1] - min(jpos), m.capacity - int(lens0.max()) - 2)
+        fresh = greedy_streams(m, pending, n, dev)
+        m.lens.copy_(lens0)
+        pending.copy_(pend0)
+        for b in range(B):
+            w = min(n, stream.shape[1] - jpos[b])
+            stream[b, jpos[b]:jpos[b] + w] = fresh[b, :w]
+    return d, a, c, left
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
 
@@ -231,6 +286,7 @@ def run_ours(args, wl, rank, world, local_rank):
         synth.planted_accepts_stratified(Ksteps, wl["mean_accept"], K, seed=1100 + 37 * rank + b)])
         for b in range(B)], axis=1)  # [total_steps, B]
     need = 1 + int(np.max(np.sum(accepts + 1, axis=0))) + K + 2  # greedy tokens the schedule reads
+    need += 4 * (K + 1)  # room for steps that leave the stream (see planted_step)
     n_var = min(Ksteps, 24) if B == 1 else 0  # the variants (batch 1) commit up to K + 1 per step
     cap = ((max(max(lens) + need + K + 2, max(lens) + (W + n_var) * (K + 1) + K + 2) + 127) // 128) * 128
 
@@ -276,14 +332,6 @@ def run_ours(args, wl, rank, world, local_rank):
         raise RuntimeError(f"device status {m.read_status()} while building the greedy stream")
     stream = stream_dev.cpu().numpy().T.copy()  # [B, need]
 
-    rng = np.random.default_rng(2000 + rank)
-    planted = np.zeros((total_steps, B, K), dtype=np.int32)
-    jpos = [0] * B
-    for t in range(total_steps):
-        for b in range(B):
-            planted[t, b] = synth.planted_drafts(stream[b], jpos[b], int(accepts[t, b]), K, V, rng)
-            jpos[b] += int(accepts[t, b]) + 1
-    planted_dev = torch.from_numpy(planted).to(dev)
     acc_all = i32(total_steps, B)
     com_all = i32(total_steps, B, K + 1)
     launches_per_step = m.launches_per_step(K)
@@ -293,6 +341,23 @@ def run_ours(args, wl, rank, world, local_rank):
     def reset():
         m.lens.copy_(lens_dev)
         pending.copy_(pend0)
+
+    # untimed rehearsal: plant every step's drafts from the greedy streams and check it on the host;
+    # the timed runs replay the same drafts from the same state and must give the same results
+    rng = np.random.default_rng(2000 + rank)
+    planted = np.zeros((total_steps, B, K), dtype=np.int32)
+    acc_ref = np.zeros((total_steps, B), dtype=np.int64)
+    com_ref = np.zeros((total_steps, B, K + 1), dtype=np.int32)
+    jpos, rebuilt = [0] * B, 0
+    stream0 = stream[:, 0].copy()
+    reset()
+    for t in range(total_steps):
+        if max(jpos) + K + 2 > stream.shape[1]:
+            raise RuntimeError("the greedy streams are too short for the planted schedule")
+        planted[t], acc_ref[t], com_ref[t], left = planted_step(m, pending, dev, stream, jpos, accepts[t], K, V, rng,
+                                                                acc_all[t], com_all[t])
+        rebuilt += int(left)
+    planted_dev = torch.from_numpy(planted).to(dev)
 
     def run_steps(lo, hi):
         for t in range(lo, hi):
@@ -327,11 +392,11 @@ def run_ours(args, wl, rank, world, local_rank):
     com = com_all.cpu().numpy()
     if m.read_status() != 0:
         err = f"device status {m.read_status()} after the timed run"
-    elif not np.array_equal(acc, accepts[:total_steps]):
-        err = "accept lengths differ from the planted schedule"
+    elif not np.array_equal(acc, acc_ref) or not np.array_equal(com, com_ref):
+        err = "the timed steps differ from the rehearsal on the same drafts"
     else:
         for b in range(B):
-            out = [int(stream[b, 0])]
+            out = [int(stream0[b])]
             for t in range(total_steps):
                 out.extend(int(x) for x in com[t, b, :max(acc[t, b], 0) + 1])
             if out != [int(x) for x in stream[b, :len(out)]]:
@@ -434,13 +499,13 @@ def run_ours(args, wl, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize(dev)
     e2e_ms = rank_reduce(e0.elapsed_time(e1), "max", world, dev)
-    raise_on_any_rank(None if np.array_equal(h_acc.numpy()[W:], accepts[W:total_steps])
+    raise_on_any_rank(None if np.array_equal(h_acc.numpy()[W:], acc_ref[W:total_steps])
                       else "end-to-end pass: accept lengths differ from the planted schedule", world, dev)
 
     variants = {}
     if B == 1:
         try:  # measured after the main line's numbers; a failure here must not cost the main line
-            variants = measure_variants(m, orthrus, dev, wl, W, Ksteps, planted_dev, accepts[:, 0], reset,
+            variants = measure_variants(m, orthrus, dev, wl, W, Ksteps, planted_dev, acc_ref[:, 0], reset,
                                         pending, cap, rank)
         except RuntimeError as e:
             variants = {"variants_error": str(e)}
@@ -464,7 +529,7 @@ def run_ours(args, wl, rank, world, local_rank):
         "launches": launches_per_step * Ksteps, "e2e_ms": e2e_ms,
         "h2d": B * K * 4, "d2h": B * 4 + B * (K + 1) * 4, "hbm_peak": hbm_peak, "tf_peak": tf_peak,
         "peak_src": peak_src, "t_gen": t_gen, "weights": w, "stream": stream[0], "accepts": acc,
-        "mean_committed": float(np.mean(acc[W:] + 1)), "cap": cap, "lens": lens,
+        "mean_committed": float(np.mean(acc[W:] + 1)), "cap": cap, "lens": lens, "rebuilt": rebuilt,
         "ar_ms": ar_ms, "ar_tokens": ar_tokens,
     }
     return res
@@ -522,12 +587,32 @@ def run_attention_bench(args, wl, rank, world, local_rank):
             one_pass()
         e1.record()
         torch.cuda.synchronize(dev)
+        eager_call = e0.elapsed_time(e1) / (Ks * L)
+        # the 36 calls of a pass as one CUDA graph: each call's host work (five tensor maps, the
+        # counter reset, the launch) is paid at capture, so the replay times the device work
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            one_pass()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        with torch.cuda.graph(graph):
+            one_pass()
+        for _ in range(W):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(Ks):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
         if int(status.item()) != 0:
             raise RuntimeError(f"attention status {int(status.item())}")
         ms = e0.elapsed_time(e1)
         per_call = ms / (Ks * L)
         modes["draft" if mode == 0 else "verify"] = {
-            "Q": Q, "keys": keys, "us_per_call": round(per_call * 1e3, 3), "bytes_per_call": call_bytes,
+            "Q": Q, "keys": keys, "us_per_call": round(per_call * 1e3, 3),
+            "us_per_call_eager": round(eager_call * 1e3, 3), "bytes_per_call": call_bytes,
             "gbs": round(call_bytes / (per_call * 1e-3) / 1e9, 1),
             "hbm_frac": round(call_bytes / (per_call * 1e-3) / 1e9 / hbm_peak, 4),
             "tflops": round(call_flops / (per_call * 1e-3) / 1e12, 2)}
@@ -540,7 +625,8 @@ def run_attention_bench(args, wl, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {"workload": args.workload, "layers_rotated": L, "cache_keys": n, "K": wl["K"],
                        "heads": H, "kv_heads": Hkv, "head_dim": d,
-                       "l2": "36 distinct layer caches per step (600 MB), larger than L2"},
+                       "l2": "36 distinct layer caches per step (600 MB), larger than L2",
+                       "launch": "one CUDA graph per step: 36 orthrus_attention calls (counter reset + kernel)"},
             "modes": modes,
             "roofline": {"kernel": "attention", "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(gbs / hbm_peak, 4), "traffic": None, "peak_source": peak_src},
@@ -567,7 +653,8 @@ def run_dynamic_k(args, wl, rank, world, local_rank):
     ks = [8, 16, 32, 64]
     Kmax = max(ks)
     n_dyn = args.steps
-    need = n_dyn * (Kmax + 1) + Kmax + 3
+    W = args.warmup
+    need = (W + n_dyn + 4) * (Kmax + 1) + Kmax + 3  # the sweep's warm-up steps, and room for rebuilt streams
     lens = prompt_lengths(wl, rank)
     cap = ((max(lens) + need + Kmax + 2 + 127) // 128) * 128
     w = synth.make_weights(shape, 1, 2)
@@ -579,45 +666,49 @@ def run_dynamic_k(args, wl, rank, world, local_rank):
     i32 = lambda *s: torch.zeros(s, dtype=torch.int32, device=dev)
     pending = i32(B)
     m.prefill(torch.from_numpy(toks).to(dev), lens, pending)
-    stream_dev = i32(need, B)
-    stream_dev[0] = pending
-    ar1, acc1 = i32(B, 1), i32(B)
-    for j in range(1, need):
-        m.verify_block(pending, None, 0, ar1)
-        m.accept_commit(pending, None, ar1, 0, acc1, stream_dev[j])
-    torch.cuda.synchronize(dev)
-    if m.read_status() != 0:
-        raise RuntimeError(f"device status {m.read_status()} while building the greedy streams")
-    stream = stream_dev.cpu().numpy().T.copy()
+    stream = greedy_streams(m, pending, need, dev)
     lens_dev = torch.tensor(lens, dtype=torch.int32, device=dev)
     pend0 = torch.from_numpy(stream[:, 0].astype(np.int32)).to(dev)
     acc = i32(B)
     coms = {K: i32(B, K + 1) for K in ks}  # committed ids [B][K + 1], one buffer per block size
 
     def run(schedule, choose, n_steps, timed_from):
-        """schedule(t, K, rng) -> accept lengths [B]; choose(stats) -> K. Returns (ms of the steps
-        from timed_from on, committed tokens there, Ks used)."""
+        """schedule(t, K, rng) -> accept lengths [B]; choose(stats) -> K. An untimed rehearsal plants
+        every step's drafts (planted_step); the timed pass replays them from the same state, reading
+        every step's accept lengths on the host for the policy, and must reproduce the rehearsal.
+        Returns (ms of the steps from timed_from on, committed tokens there, Ks used)."""
+        st = stream.copy()
         m.lens.copy_(lens_dev)
         pending.copy_(pend0)
         rng = np.random.default_rng(7000 + rank)
         stats = orthrus.accept_stats(B)
-        jpos = [0] * B
+        jpos, rec = [0] * B, []
+        for t in range(n_steps):
+            K = choose(stats)
+            a_plan = schedule(t, K, rng)
+            if max(jpos) + K + 2 > st.shape[1]:
+                raise RuntimeError("the greedy streams are too short for the planted schedule")
+            d, a, _, _ = planted_step(m, pending, dev, st, jpos, a_plan, K, V, rng, acc, coms[K])
+            orthrus.accept_stats_update(stats, a.tolist(), K, 0.7)
+            rec.append((K, torch.from_numpy(d).to(dev), a))
+        m.lens.copy_(lens_dev)
+        pending.copy_(pend0)
+        stats = orthrus.accept_stats(B)
         used, tokens = [], 0
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
         for t in range(n_steps):
             if t == timed_from:
                 torch.cuda.synchronize(dev)
                 e0.record()
             K = choose(stats)
-            a_plan = schedule(t, K, rng)
-            d = np.stack([synth.planted_drafts(stream[b], jpos[b], int(a_plan[b]), K, V, rng) for b in range(B)])
-            m.decode_step(pending, K, torch.from_numpy(d.astype(np.int32)).to(dev), acc, coms[K])
+            if K != rec[t][0]:
+                raise RuntimeError(f"step {t}: the policy chose K = {K}, the rehearsal {rec[t][0]}")
+            m.decode_step(pending, K, rec[t][1], acc, coms[K])
             a = acc.cpu().numpy()  # the policy reads every step's accept lengths on the host
-            if not np.array_equal(a, a_plan):
-                raise RuntimeError(f"step {t}, K = {K}: accept lengths {a} differ from the planted {a_plan}")
+            if not np.array_equal(a, rec[t][2]):
+                raise RuntimeError(f"step {t}, K = {K}: accept lengths {a} differ from the rehearsal {rec[t][2]}")
             orthrus.accept_stats_update(stats, a.tolist(), K, 0.7)
-            for b in range(B):
-                jpos[b] += int(a[b]) + 1
             if t >= timed_from:
                 tokens += int(np.sum(a + 1))
                 used.append(K)
@@ -627,7 +718,6 @@ def run_dynamic_k(args, wl, rank, world, local_rank):
             raise RuntimeError(f"device status {m.read_status()}")
         return e0.elapsed_time(e1), tokens, used
 
-    W = args.warmup
     # 1. the sweep: step time and tok/s of each K on its own planted schedule (accept mean K / 5)
     sweep, step_ms = {}, []
     for K in ks:
@@ -921,6 +1011,7 @@ def main():
                    "prompt": wl["prompt"] if "prompt" in wl else f"{min(r['lens'])}..{max(r['lens'])} tokens",
                    "K": wl["K"], "planted_mean_accept": wl["mean_accept"], "capacity": r["cap"],
                    "planted_schedule": "stratified quantiles of the capped geometric law, seeded order",
+                   "streams_rebuilt": r["rebuilt"],
                    "tokens_per_step_expected": round(synth.capped_geometric_mean(wl["mean_accept"], wl["K"]) + 1, 4),
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (30.3 GB of weights streamed per step)"},

@@ -314,9 +314,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       } else {
         const int slot = bh * a.row_tiles + rt;
-        float* po = a.part_o + (((size_t)slot * a.max_chunks + chunk) * 128 + r) * d;
+        // partial O as [chunk][d/4][128 rows][4]: a warp's float4 stores (and the merge's
+        // loads) are 512 contiguous bytes
+        float4* po = reinterpret_cast<float4*>(a.part_o) + ((size_t)slot * a.max_chunks + chunk) * (d / 4) * 128 + r;
 #pragma unroll
-        for (int e = 0; e < d; e += 4) *reinterpret_cast<float4*>(po + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        for (int e = 0; e < d; e += 4) po[(size_t)(e / 4) * 128] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         a.part_ml[((size_t)slot * a.max_chunks + chunk) * 128 + r] = make_float2(m_run, l_run);
         __threadfence();
         named_bar_sync(1, 128);
@@ -329,33 +331,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           __threadfence();
           if (threadIdx.x == 64) a.counter[slot] = 0;
           if (row_ok) {
+            // chunks merged in chunk order; the weights first, then O in 64-column halves
+            // with two chunks' loads in flight
+            const float2* ml_row = a.part_ml + (size_t)slot * a.max_chunks * 128 + r;
             float mstar = -INFINITY;
-            for (int cc = 0; cc < n_chunks; ++cc)
-              mstar = fmaxf(mstar, __ldcg(&a.part_ml[((size_t)slot * a.max_chunks + cc) * 128 + r].x));
+            for (int cc = 0; cc < n_chunks; ++cc) mstar = fmaxf(mstar, __ldcg(ml_row + (size_t)cc * 128).x);
             float L = 0.f;
-#pragma unroll
-            for (int e = 0; e < d; ++e) o[e] = 0.f;
             for (int cc = 0; cc < n_chunks; ++cc) {
-              const float2 ml = __ldcg(&a.part_ml[((size_t)slot * a.max_chunks + cc) * 128 + r]);
-              const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mstar);
-              L += ml.y * w;
-              const float* pc = a.part_o + (((size_t)slot * a.max_chunks + cc) * 128 + r) * d;
-#pragma unroll
-              for (int e = 0; e < d; e += 4) {
-                const float4 x = __ldcg(reinterpret_cast<const float4*>(pc + e));
-                o[e] += x.x * w;
-                o[e + 1] += x.y * w;
-                o[e + 2] += x.z * w;
-                o[e + 3] += x.w * w;
-              }
+              const float2 ml = __ldcg(ml_row + (size_t)cc * 128);
+              L += ml.y * ((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mstar));
             }
             const float inv = L > 0.f ? 1.f / L : 0.f;
+            const float4* p4 = reinterpret_cast<const float4*>(a.part_o) + (size_t)slot * a.max_chunks * (d / 4) * 128 + r;
+#pragma unroll 1
+            for (int h = 0; h < d / 64; ++h) {
+              float acc[64];
 #pragma unroll
-            for (int e = 0; e < d; e += 8) {
-              float y8[8];
+              for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+#pragma unroll 2
+              for (int cc = 0; cc < n_chunks; ++cc) {
+                const float2 ml = __ldcg(ml_row + (size_t)cc * 128);
+                const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mstar);
+                const float4* pc = p4 + ((size_t)cc * (d / 4) + h * 16) * 128;
 #pragma unroll
-              for (int t = 0; t < 8; ++t) y8[t] = o[e + t] * inv;
-              st_split_x8(dst + e, dst + a.out_lo + e, y8);
+                for (int e = 0; e < 16; ++e) {
+                  const float4 x = __ldcg(pc + (size_t)e * 128);
+                  acc[4 * e] += x.x * w;
+                  acc[4 * e + 1] += x.y * w;
+                  acc[4 * e + 2] += x.z * w;
+                  acc[4 * e + 3] += x.w * w;
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 64; e += 8) {
+                float y8[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) y8[t] = acc[e + t] * inv;
+                st_split_x8(dst + h * 64 + e, dst + a.out_lo + h * 64 + e, y8);
+              }
             }
           }
         }

@@ -106,6 +106,7 @@ constexpr int kMaxChunks = 34;        // key chunks per slot (32 cache chunks + 
 constexpr int kCombineRows = 16;      // rows per merge unit
 constexpr int kScratchBytes = 19584;  // P tile (16 KB) / epilogue staging (36 x 132 fp32 + sums), shared
 constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers
+constexpr float kRescaleLog2 = 8.f;   // attention: largest log2 step of a score over the exponent offset
 
 struct LayerNorms {  // device-resident per-layer gains (fp32)
   const float *attn_norm, *mlp_norm, *q_norm, *k_norm, *wd_q_norm, *wd_k_norm;
@@ -213,7 +214,12 @@ __host__ inline size_t fwd_fixed_smem(int d) {
 }
 // ring stage: 32 KB weight box (128 rows x two k chunks) + activation box (Mt rows x two k
 // chunks x two planes; the LM head reads the hi plane only)
-__host__ inline size_t fwd_stage_bytes(int Mt) { return 32768 + (size_t)Mt * 512; }
+// In attention phases a stage holds one 64-key tile: K, V (64 x d fp16 each) and its P tile
+// (128 rows x 64 keys fp16).
+__host__ __device__ inline uint32_t fwd_stage_bytes(int Mt, int d) {
+  const uint32_t proj = 32768u + (uint32_t)Mt * 512u, att = 2u * 128u * (uint32_t)d + 16384u;
+  return proj > att ? proj : att;
+}
 
 // Shared state every role derives identically at kernel start.
 struct FwdGeom {
@@ -1291,10 +1297,12 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
         }
         if (!row_ok) lim = t.key_lo;
         // O accumulates in TMEM across the unit's key tiles (P V MMAs with accumulate);
-        // when a row's running maximum moves, the row of O is rescaled in TMEM before
-        // the next P V. O is read into registers once, after the last tile.
+        // when a row's exponent offset moves (below), the row of O is rescaled in TMEM
+        // before the next P V. O is read into registers once, after the last tile. P of a
+        // tile sits beside its V in the ring stage, so P of the next tile can be written
+        // while this tile's P V still reads.
         float m_run = -INFINITY, l_run = 0.f;
-        for (int j = 0; j < t.tiles; ++j, it += 2, ++ta) {
+        for (int j = 0; j < t.tiles; ++j, ++it, ++ta) {
           // score buffer ta & 1; its barrier completes once per use, every second tile
           if (!bar_wait_all(&s_full[(ta & 1) * 3], (uint32_t)(ta >> 1) & 1u, 14)) {
             ok = false;
@@ -1323,12 +1331,19 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
             }
           }
           const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * a.scale_log2;
-          const float m_new = fmaxf(m_run, mx);
-          const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+          // The exponent offset m_run moves only when a score passes it by more than
+          // kRescaleLog2 (then the weights below stay under 2^kRescaleLog2, well inside fp16),
+          // so O is rarely rescaled and this tile's softmax need not wait for the previous P V.
+          const bool grow = mx > m_run + kRescaleLog2;
+          const float m_new = grow ? mx : m_run;
+          const float alpha = (grow && m_run != -INFINITY) ? fast_exp2(m_run - m_new) : 1.f;
           if (j == 0 && et == 0) tl_mark<TL>(a, n_ph, p, TL_S_PART);  // row maxima done
-          if (j > 0) {
+          // this tile's stage: K, V, then P. Its K and V landed before S was issued, and the
+          // P region's previous reader released the stage before they were loaded.
+          const int vs = it % S;
+          if (j > 0 && named_bar_or(1, 128, alpha != 1.f)) {
             // the previous tile's P V must be complete before O is rescaled
-            if (!bar_wait_all(o_full, (uint32_t)(ta - 1) & 1u, 15)) {
+            if (!bar_wait_all(&o_full[(ta - 1) & 1], (uint32_t)((ta - 1) >> 1) & 1u, 15)) {
               ok = false;
               break;
             }
@@ -1344,6 +1359,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               }
             }
           }
+          uint8_t* vb = smem + (size_t)vs * stage_bytes + halves * 8192;  // V, then P
           float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
           for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -1360,7 +1376,7 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
               __half2 h2 = __floats2half2_rn(p0, p1);
               pk[tt / 2] = *reinterpret_cast<uint32_t*>(&h2);
             }
-            uint8_t* rowp = scr + row * 128;
+            uint8_t* rowp = vb + halves * 8192 + row * 128;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               const int ch = (c0 >> 3) + q4;
@@ -1370,28 +1386,26 @@ __device__ __forceinline__ void fwd_epilogue_role(const FwdArgs& a, const FwdGeo
           }
           l_run = l_run * alpha + (sum0 + sum1);
           m_run = m_new;
-          // V rows of keys no row may see are zeroed (stale or poisoned cache rows)
-          if (key0 + 64 > kv_end && row < 64 && key0 + row >= kv_end) {
-            const int vs = (it + 1) % S;
-            if (mbar_wait_abortable(&full[vs], (uint32_t)((it + 1) / S) & 1u, a.status)) {
-              uint8_t* vb = smem + (size_t)vs * stage_bytes;
+          // V rows of keys no row may see are zeroed (stale or poisoned cache rows); the wait
+          // orders these writes after the TMA's
+          if (key0 + 64 > kv_end && row < 64 && key0 + row >= kv_end &&
+              mbar_wait_abortable(&full[vs], (uint32_t)(it / S) & 1u, a.status)) {
 #pragma unroll
-              for (int hh = 0; hh < halves; ++hh) {
-                uint4* vr = reinterpret_cast<uint4*>(vb + hh * 8192 + row * 128);
+            for (int hh = 0; hh < halves; ++hh) {
+              uint4* vr = reinterpret_cast<uint4*>(vb + hh * 8192 + row * 128);
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) vr[q8] = make_uint4(0u, 0u, 0u, 0u);
-              }
+              for (int q8 = 0; q8 < 8; ++q8) vr[q8] = make_uint4(0u, 0u, 0u, 0u);
             }
           }
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(p_full);
+          if (lane == 0) mbar_arrive(&p_full[ta & 1]);
           if (j == 0 && et == 0) tl_mark<TL>(a, n_ph, p, TL_S_CNT);  // P written
         }
         if (!ok) break;
         // the unit's last P V, then O into registers
-        if (!bar_wait_all(o_full, (uint32_t)(ta - 1) & 1u, 15)) {
+        if (!bar_wait_all(&o_full[(ta - 1) & 1], (uint32_t)((ta - 1) >> 1) & 1u, 15)) {
           ok = false;
           break;
         }
@@ -1513,8 +1527,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   constexpr int d = D_HEAD;
   constexpr int halves = d / 64;
   const int S = a.stages;
-  const uint32_t x_bytes = (uint32_t)a.Mt * 512u;  // two k chunks x two planes of Mt rows
-  const uint32_t stage_bytes = 32768u + x_bytes;
+  const uint32_t stage_bytes = fwd_stage_bytes(a.Mt, d);
   uint8_t* sQ = smem + (size_t)S * stage_bytes;   // attention Q tile, d/64 blocks of 128 rows x 64
   uint8_t* scr = sQ + (size_t)128 * d * 2;         // P tile / epilogue staging
   unsigned long long* red = (unsigned long long*)(scr + kScratchBytes);
@@ -1528,12 +1541,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   uint64_t* accf = bars + 2 * kMaxStages;  // [2]
   uint64_t* acce = accf + 2;               // [2]
   uint64_t* s_full = acce + 2;  // [0] and [3]: scores of even / odd key tiles ready
-  uint64_t* p_full = s_full + 1;
-  uint64_t* o_full = s_full + 2;
   uint64_t* done = s_full + 4;
   uint64_t* q_full = s_full + 5;
   uint64_t* q_empty = s_full + 6;
-  uint32_t* tmem_slot = (uint32_t*)(q_empty + 1);
+  uint64_t* p_full = s_full + 7;  // [2]: P of even / odd key tiles written
+  uint64_t* o_full = s_full + 9;  // [2]: P V of even / odd key tiles done
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 11);
   int* flag = (int*)(tmem_slot + 1);  // [8]
   FwdGeom* geom_s = (FwdGeom*)(flag + 8);
 
@@ -1554,8 +1567,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
     }
     mbar_init(s_full, 1);
     mbar_init(s_full + 3, 1);  // second score buffer
-    mbar_init(p_full, 4);
-    mbar_init(o_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&p_full[b], 4);
+      mbar_init(&o_full[b], 1);
+    }
     mbar_init(done, 1);
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
@@ -1563,22 +1578,40 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   }
   if (threadIdx.x < a.nb) lens_s[threadIdx.x] = a.len[threadIdx.x];
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     FwdGeom g;
     g.rows_per_slot = a.Q * a.G;
     g.rt = (g.rows_per_slot + 127) / 128;
     g.slots = a.nb * a.Hkv * g.rt;
     g.CK = a.ck;
-    slot_pre[0] = 0;
-    bool multi = false;
-    for (int s = 0; s < g.slots; ++s) {
-      const int ch = slot_chunks(a, g, lens_s, s);
-      multi = multi || ch > 1;
-      slot_pre[s + 1] = slot_pre[s] + ch;
+    if (a.view == VIEW_DRAFT) {
+      // The verify view keeps the plan's chunk length, so that its rows and plain decoding
+      // see the same chunk boundaries. The draft view's rows are matched with no other
+      // launch, so its chunks are the shortest whose units (one per chunk, plus the block)
+      // fit one wave of CTAs for the current cache lengths: lane j tries ck0 + 64 j.
+      int n_max = 0;
+      for (int bb = lane; bb < a.nb; bb += 32) n_max = max(n_max, min(lens_s[bb], a.cap));
+      for (int o = 16; o > 0; o >>= 1) n_max = max(n_max, __shfl_xor_sync(0xffffffffu, n_max, o));
+      const int ck0 = max(64, ((n_max + 31) / 32 + 63) / 64 * 64);  // at most 32 cache chunks
+      const int ck = ck0 + 64 * lane;
+      long long units = 0;
+      for (int bb = 0; bb < a.nb; ++bb)
+        units += (long long)a.Hkv * g.rt * ((min(lens_s[bb], a.cap) + ck - 1) / ck + 1);
+      const unsigned fit = __ballot_sync(0xffffffffu, ck < a.ck && units <= Gd);
+      if (fit) g.CK = ck0 + 64 * (__ffs((int)fit) - 1);
     }
-    g.att_units = slot_pre[g.slots];
-    g.comb_units = multi ? g.slots * (128 / kCombineRows) : 0;
-    *geom_s = g;
+    if (lane == 0) {
+      slot_pre[0] = 0;
+      bool multi = false;
+      for (int s = 0; s < g.slots; ++s) {
+        const int ch = slot_chunks(a, g, lens_s, s);
+        multi = multi || ch > 1;
+        slot_pre[s + 1] = slot_pre[s] + ch;
+      }
+      g.att_units = slot_pre[g.slots];
+      g.comb_units = multi ? g.slots * (128 / kCombineRows) : 0;
+      *geom_s = g;
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -1675,11 +1708,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
             const AttUnit t = att_unit(a, g, lens_s, slot_pre, u);
             const int zc = (l * a.batch + t.bb) * a.Hkv + t.kvh;
             const int qrow = (t.bb * a.Hkv + t.kvh) * g.rows_per_slot + t.r * 128;
-            const int n_loads = 2 * t.tiles;
             // Cache keys below len were written by earlier launches: their K/V tiles are
             // loaded without waiting for this layer's q/k/v phase. The Q tile and block
             // keys wait for it; Q goes out before the first such load, or after the first
-            // K/V pair when that pair is independent.
+            // K/V tile when that tile is independent.
             bool q_issued = false;
             auto issue_q = [&]() -> bool {
               if (!dep_ready(dep)) return false;
@@ -1697,11 +1729,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 break;
               }
             }
-            for (int j = 0; j < n_loads; ++j, ++it) {
-              const int key0 = t.key_lo + (j >> 1) * 64;
-              // Q before any wait that needs this unit's own S MMAs (with two ring stages
-              // the stage of load j = 2 is that of load 0)
-              if (!wprod && (j >= 2 || !independent(key0)) && !q_issued && !issue_q()) {
+            for (int j = 0; j < t.tiles; ++j, ++it) {
+              const int key0 = t.key_lo + j * 64;
+              // Q before any wait that may need this unit's own S MMAs (a later tile's stage
+              // can be one this unit's first tile frees)
+              if (!wprod && (j >= 1 || !independent(key0)) && !q_issued && !issue_q()) {
                 ok = false;
                 break;
               }
@@ -1722,11 +1754,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
                 ok = false;
                 break;
               }
+              // K and V of the tile into one stage: K at 0, V at 128 d bytes (P follows them)
               uint8_t* st = stage_ptr(s);
-              const bool is_v = j & 1;
-              const CUtensorMap* mp = t.blk ? (is_v ? gm + G_VB64 : gm + G_KB64) : (is_v ? gm + G_VC64 : gm + G_KC64);
-              mbar_arrive_expect_tx(&full[s], 8192u * halves);
-              for (int hh = 0; hh < halves; ++hh) tma_load_3d(st + hh * 8192, mp, &full[s], hh * 64, key0, zc);
+              const CUtensorMap* mk = t.blk ? gm + G_KB64 : gm + G_KC64;
+              const CUtensorMap* mv = t.blk ? gm + G_VB64 : gm + G_VC64;
+              mbar_arrive_expect_tx(&full[s], 16384u * halves);
+              for (int hh = 0; hh < halves; ++hh) tma_load_3d(st + hh * 8192, mk, &full[s], hh * 64, key0, zc);
+              for (int hh = 0; hh < halves; ++hh)
+                tma_load_3d(st + (halves + hh) * 8192, mv, &full[s], hh * 64, key0, zc);
             }
             if (ok && !wprod && !q_issued && !issue_q()) {
               ok = false;
@@ -1751,7 +1786,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
       const uint32_t idesc_g2 = idesc_bf16(128, 2 * a.Mt, false);  // hi rows then lo rows
       const uint32_t idS = idesc_f16(128, 64, false);  // fp16 q and K
       const uint32_t idO = idesc_f16(128, d, true);    // fp16 P and V
-      const uint32_t pa = smem_u32(scr);
       int it = 0, seg = 0, ta = 0, qu = 0;
       bool ok = true;
       for (int p = 0; ok && p < n_ph; ++p) {
@@ -1836,8 +1870,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               for (int kk = 0; kk < d / 16; ++kk)
                 mma_ss(ts, qd0 + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                        kd0 + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
-              mma_commit(&s_full[(taj & 1) * 3]);
-              mma_commit(&empty[ks]);
+              mma_commit(&s_full[(taj & 1) * 3]);  // the stage is released after P V
               if (jj == t.tiles - 1) mma_commit(q_empty);  // last read of this unit's Q tile
               return true;
             };
@@ -1845,33 +1878,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
               ok = false;
               break;
             }
-            for (int j = 0; ok && j < t.tiles; ++j, it += 2, ++ta) {
-              const int vs = (it + 1) % S;
+            for (int j = 0; ok && j < t.tiles; ++j, ++it, ++ta) {
+              const int vs = it % S;  // this tile's stage (K, V and P); its full barrier was awaited for S
               // the next tile's scores go into the other buffer while the softmax warps work on
               // this one (its previous contents, tile j - 1, were read before P of j - 1)
-              if (j + 1 < t.tiles && !issue_s(j + 1, it + 2, ta + 1)) {
+              if (j + 1 < t.tiles && !issue_s(j + 1, it + 1, ta + 1)) {
                 ok = false;
                 break;
               }
-              // P of this tile written (and O rescaled) by the softmax warps, V landed
-              r = mbar_wait_code(p_full, (uint32_t)ta & 1u, a.status);
-              if (r == 1) {
-                r = mbar_wait_code(&full[vs], (uint32_t)((it + 1) / S) & 1u, a.status);
-                if (r != 1) fwd_diag(a, r, 10, p, it, vs);
-              } else {
-                fwd_diag(a, r, 9, p, it, ta);
-              }
+              // P of this tile written (and O rescaled) by the softmax warps
+              r = mbar_wait_code(&p_full[ta & 1], (uint32_t)(ta >> 1) & 1u, a.status);
               if (r != 1) {
+                fwd_diag(a, r, 9, p, it, ta);
                 ok = false;
                 break;
               }
               tc_fence_after();
-              const uint32_t va = smem_u32(stage_ptr(vs));
+              const uint32_t va = smem_u32(stage_ptr(vs)) + (uint32_t)halves * 8192u, pa = va + (uint32_t)halves * 8192u;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_ss(tO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, 8192, 1024), idO,
                             (j > 0 || kk > 0) ? 1u : 0u);
-              mma_commit(o_full);
+              mma_commit(&o_full[ta & 1]);
               mma_commit(&empty[vs]);
             }
             if (!ok) break;

@@ -439,7 +439,7 @@ GemmArgs base_gemm_args(const Plan* P) {
 // Blocks whose token rows fit two ring stages (at most 96 rows at head_dim 128) run through
 // it; larger blocks take the per-op kernels.
 bool fwd_rows_fit(int M, int d) {
-  return M <= 128 && fwd_fixed_smem(d) + 2 * fwd_stage_bytes(round_up(M, 16)) <= kSmemLimit;
+  return M <= 128 && fwd_fixed_smem(d) + 2 * (size_t)fwd_stage_bytes(round_up(M, 16), d) <= kSmemLimit;
 }
 
 bool persistent_ok(const Plan* P, int Q) {
@@ -485,7 +485,7 @@ orthrus_status launch_forward(const Plan* P, int view, int Q, const int* pending
   a.M = P->B * Q;
   a.Mt = round_up(a.M, 16);
   a.mt_idx = a.Mt / 16 - 1;
-  const size_t stage = fwd_stage_bytes(a.Mt);
+  const size_t stage = fwd_stage_bytes(a.Mt, a.d);
   // 3-4 stages of 32 KB weight boxes (96-128 KB in flight per SM): a bare TMA stream of
   // such boxes measured fastest at 4; deeper rings put more requests in flight than HBM
   // serves efficiently
@@ -827,7 +827,8 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
     const int G = cfg->n_heads / cfg->n_kv_heads;
     const int slots_v = P->B * cfg->n_kv_heads * ((G * (max_block + 1) + 127) / 128);
     const int sms = num_sms();
-    P->fwd_ck = std::max(P->fwd_ck, round_up((int)(((long long)P->cap * slots_v + sms - 1) / sms), 64));
+    const int per_slot = std::max(1, sms / std::max(1, slots_v));  // chunks per slot in one wave
+    P->fwd_ck = std::max(P->fwd_ck, round_up((P->cap + per_slot - 1) / per_slot, 64));
   }
   P->fwd_att_o = (float*)(base + wl.fwd_att_o);
   P->fwd_att_ml = (float2*)(base + wl.fwd_att_ml);
