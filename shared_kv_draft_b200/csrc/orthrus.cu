@@ -279,12 +279,23 @@ struct WsLayout {
   int chunk_keys, attn_slots, ss_ld, mega_slots;
 };
 
+bool fwd_rows_fit(int M, int d);
+
+// Largest block (token rows per sequence, at most max_block + 1) whose B rows the persistent
+// forward kernel runs; 0 if none. Larger blocks of the same plan take the per-op kernels.
+int persistent_q_max(const orthrus_config* c, int B, int max_block) {
+  for (int Q = max_block + 1; Q >= 1; --Q)
+    if (fwd_rows_fit(B * Q, c->head_dim)) return Q;
+  return 0;
+}
+
 // Attention slots of the persistent forward kernel for this batch and block limit
-// (0 when the kernel cannot run these sizes: more than 128 token rows or too many slots).
+// (0 when the kernel runs no block of this plan: too many token rows or too many slots).
 int mega_slots(const orthrus_config* c, int B, int max_block) {
   const int G = c->n_heads / c->n_kv_heads;
-  if (B * (max_block + 1) > 128 || c->d_model > 8192) return 0;
-  const int rt = (G * (max_block + 1) + 127) / 128;
+  const int qp = persistent_q_max(c, B, max_block);
+  if (qp == 0 || c->d_model > 8192) return 0;
+  const int rt = (G * qp + 127) / 128;
   const int slots = B * c->n_kv_heads * rt;
   return slots <= kMaxSlots ? slots : 0;
 }
@@ -825,7 +836,8 @@ orthrus_status orthrus_plan_init(void* plan, size_t plan_bytes, const orthrus_co
   P->fwd_ck = std::max(64, round_up((P->cap + kMaxChunks - 3) / (kMaxChunks - 2), 64));
   {
     const int G = cfg->n_heads / cfg->n_kv_heads;
-    const int slots_v = P->B * cfg->n_kv_heads * ((G * (max_block + 1) + 127) / 128);
+    const int qp = std::max(1, persistent_q_max(cfg, P->B, max_block));  // largest persistent block
+    const int slots_v = P->B * cfg->n_kv_heads * ((G * qp + 127) / 128);
     const int sms = num_sms();
     const int per_slot = std::max(1, sms / std::max(1, slots_v));  // chunks per slot in one wave
     P->fwd_ck = std::max(P->fwd_ck, round_up((P->cap + per_slot - 1) / per_slot, 64));
