@@ -104,7 +104,7 @@ constexpr int kMaxStages = 16;
 constexpr int kMaxSlots = 256;        // attention (sequence, kv head, row tile) slots per launch
 constexpr int kMaxChunks = 34;        // key chunks per slot (32 cache chunks + draft block + slack)
 constexpr int kCombineRows = 16;      // rows per merge unit
-constexpr int kScratchBytes = 19584;  // P tile (16 KB) / epilogue staging (36 x 132 fp32 + sums), shared
+constexpr int kScratchBytes = 19584;  // epilogue staging (36 x 132 fp32 + per-quarter sums)
 constexpr int kMaxGrid = 256;         // CTAs (one per SM) the unit-range table covers
 constexpr float kRescaleLog2 = 8.f;   // attention: largest log2 step of a score over the exponent offset
 
@@ -205,8 +205,8 @@ __host__ __device__ inline int fwd_phase_kind(int p, int L) {
 __host__ __device__ inline int fwd_phase_layer(int p) { return (p - 1) / kPhasesPerLayer; }
 
 // Shared memory outside the ring: the attention Q tile (128 rows x d, resident for
-// a whole attention unit, so it cannot live in the ring), the P tile / epilogue
-// staging, small per-CTA tables and the barriers.
+// a whole attention unit, so it cannot live in the ring), the epilogue staging, small
+// per-CTA tables and the barriers. (Attention's P tiles live in the ring stages.)
 __host__ inline size_t fwd_fixed_smem(int d) {
   return 1024 /*align*/ + (size_t)128 * d * 2 /*Q*/ + kScratchBytes + 144 * 8 /*red*/ + 128 * 4 /*rstd*/ +
          128 * 4 /*lens*/ + (kMaxSlots + 1) * 4 /*slot prefix*/ + 64 * 8 /*barriers*/ + 64 * 4 /*misc*/ +
@@ -1529,7 +1529,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) forward_kernel(const __grid_co
   const int S = a.stages;
   const uint32_t stage_bytes = fwd_stage_bytes(a.Mt, d);
   uint8_t* sQ = smem + (size_t)S * stage_bytes;   // attention Q tile, d/64 blocks of 128 rows x 64
-  uint8_t* scr = sQ + (size_t)128 * d * 2;         // P tile / epilogue staging
+  uint8_t* scr = sQ + (size_t)128 * d * 2;         // epilogue staging
   unsigned long long* red = (unsigned long long*)(scr + kScratchBytes);
   float* rstd_s = (float*)(red + 144);
   int* lens_s = (int*)(rstd_s + 128);
