@@ -224,7 +224,8 @@ def greedy_streams(m, pending, n, dev):
     for j in range(1, n):
         m.verify_block(pending, None, 0, ar1)
         m.accept_commit(pending, None, ar1, 0, acc1, sd[j])
-    torch.cuda.synchronize(dev)
+    if torch.device(dev).type == "cuda":
+        torch.cuda.synchronize(dev)
     if m.read_status() != 0:
         raise RuntimeError(f"device status {m.read_status()} while building the greedy streams")
     return sd.cpu().numpy().T.copy()
