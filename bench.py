@@ -643,7 +643,8 @@ def run_dynamic_k(args, wl, rank, world, local_rank):
          phase (0.95) and an open-ended one (0.6), every 8 steps, is run with each fixed K
          and with the policy (orthrus_choose_block_size, fed every step by the host copy of
          the accept lengths), on the same seeded draws. Drafts are planted from each
-         sequence's greedy stream; every run must commit exactly the planted prefixes."""
+         sequence's greedy stream (rebuilt where a verify block on the per-op kernels breaks a
+         near tie differently, see planted_step); every timed run must reproduce its rehearsal."""
     import torch
 
     from shared_kv_draft_b200 import orthrus
