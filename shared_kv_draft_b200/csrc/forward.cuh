@@ -1,8 +1,9 @@
 // Persistent forward kernel: one launch runs a whole draft-view or verify-view
 // forward of the Orthrus decode step (embedding, every layer's q/k/v
 // projection, block attention, output projection, SwiGLU MLP, final norm, LM
-// head and argmax) for a block of at most 128 token rows, and the verify launch
-// also runs the greedy consensus and KV commit at its end.
+// head and argmax) for a block whose token rows fit two ring stages (at most 96 at
+// head dim 128), and the verify launch also runs the greedy consensus and KV commit
+// at its end.
 //
 // Why one kernel: at decode sizes every projection is a weight stream of 5-30
 // microseconds, so separate launches pay a start-up and a split-K tail per
@@ -33,8 +34,10 @@
 // logits' error, so the operands carry more bits than bf16:
 //   - an activation that feeds a layer projection (xg, the attention output, the SwiGLU
 //     output) is written as two bf16 planes, hi = bf16(x) and lo = bf16(x - hi); every
-//     weight chunk is multiplied with both (two MMAs into one fp32 accumulator), so the
-//     projection sees x to about 2^-17 relative. The LM head reads the hi plane only;
+//     weight chunk is multiplied with both in one MMA (N = 2 Mt: the hi rows, then the lo
+//     rows; the two fp32 accumulators sit side by side in TMEM and the epilogue adds
+//     them), so the projection sees x to about 2^-17 relative. The LM head reads the hi
+//     plane only;
 //   - attention runs on fp16 operands: q and the softmax weights P (11 significant bits),
 //     and K/V, bf16 values held in the fp16 encoding.
 //
@@ -43,9 +46,9 @@
 // 1 = tcgen05.mma issuer, warps 2-5 = epilogue (TMEM -> registers -> fused
 // epilogue), attention softmax, embedding and chunk merge. Two issuing threads
 // matter: one thread issuing 8 KB copies streams about 4 TB/s, two reach the
-// HBM rate. Ring stage = a 32 KB slot (a weight box of 128 rows x two 64-wide k
-// chunks, or an attention K / V tile) + an activation slot of Mt rows x two k chunks x
-// two planes.
+// HBM rate. Ring stage = a 32 KB weight box (128 rows x two 64-wide k chunks) + an
+// activation box of Mt rows x two k chunks x two planes; in attention phases a stage
+// holds one 64-key tile's K, V and P tile instead.
 #pragma once
 #include "gemm.cuh"
 
