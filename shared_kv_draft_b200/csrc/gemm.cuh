@@ -22,8 +22,9 @@
 //    cache (or the draft block scratch), SwiGLU (each tile holds 64 gate rows
 //    and the 64 matching up rows; hi and lo planes out), and LM-head argmax
 //    (64-bit max of (value, -index)).
-//  * X may come in two bf16 planes (hi + lo of one fp32 activation): each
-//    weight chunk is multiplied with both into the same fp32 accumulator.
+//  * X may come in two bf16 planes (hi + lo of one fp32 activation): one MMA
+//    per k slice multiplies the weight chunk with both (N = 2 Mt), into two fp32
+//    accumulators side by side in TMEM that the epilogue adds.
 #pragma once
 #include "ptx.cuh"
 
@@ -55,7 +56,7 @@ struct GemmArgs {
   int m_tiles, n_tiles, k_chunks;
   long long total_units;
   int stages;
-  int planes;                // activation planes of X: 2 (hi + lo, two MMAs per chunk) or 1
+  int planes;                // activation planes of X: 2 (hi + lo rows in one MMA of N = 2 Mt) or 1
   int swiglu_F;              // SwiGLU: row offset of the up rows in W
   float* partial;            // [2 * grid][128 rows][Mt] fp32 partial sums of split tiles
   int* tile_counter;         // [m_tiles * n_tiles], zero between launches
