@@ -179,17 +179,21 @@ enum {
  * Host memory of `kinds` and `count` must stay valid while the hook is set. */
 orthrus_status orthrus_trace(void* plan, void* const* events, int32_t* kinds, int32_t capacity, int32_t* count);
 
-/* Profiling hook of the persistent forward kernel (the draft and verify views
- * when batch * (K + 1) <= 128). While set, every launch of it writes, for each
- * CTA c and phase p (p = 0 embedding, 1 + 6 l + {0..5} = layer l's q/k/v
- * projection, attention, chunk merge, output projection, gate/up, down,
- * 1 + 6 L = LM head), eight globaltimer stamps (ns, uint64) at
- * device_buf[(c * (2 + 6 L) + p) * 8 + e]: e = 0/1 first/last weight load
+/* Profiling hook of the persistent forward kernel (the draft and verify views of
+ * blocks whose token rows fit it: at most 96 at head dim 128). While set, every
+ * launch of it writes, for each CTA c and phase p (p = 0 embedding, 1 + 6 l +
+ * {0..5} = layer l's q/k/v projection, attention, chunk merge, output projection,
+ * gate/up, down, 1 + 6 L = LM head), sixteen globaltimer stamps (ns, uint64) at
+ * device_buf[(c * (2 + 6 L) + p) * 16 + e]: e = 0/1 first/last weight load
  * issued, 2/3 activation dependency met/last activation load issued, 4/5 first
- * MMA/last MMA commit, 6/7 epilogue dependency met/phase finished. Entries of
- * events that did not occur keep their previous contents. device_buf: device
- * memory of at least orthrus_timeline_bytes(plan) bytes, owned by the caller;
- * NULL switches the hook off. */
+ * MMA/last MMA commit, 6/7 epilogue dependency met/phase finished; for the last
+ * epilogue segment of a projection phase 8..13 = accumulator ready, partial stored,
+ * arrival counted, partials loaded, epilogue done, completion signalled; in an
+ * attention phase 14/15 = first score tile ready, O read (9/10 row maxima done and
+ * P written for the first tile, 8 later score tiles ready). Entries of events that
+ * did not occur keep their previous contents. device_buf: device memory of at least
+ * orthrus_timeline_bytes(plan) bytes, owned by the caller; NULL switches the hook
+ * off. */
 size_t orthrus_timeline_bytes(const void* plan);
 orthrus_status orthrus_timeline(void* plan, void* device_buf, size_t bytes);
 
