@@ -1,6 +1,6 @@
 """Phase timeline of the persistent forward kernel (profiling tool).
 
-    python -m shared_kv_draft_b200.timeline [--layers L] [--K 32] [--prompt 512] [--reps 3]
+    python -m shared_kv_draft_b200.timeline [--layers L] [--K 32] [--prompt 512] [--capacity 1792] [--reps 3]
 
 Builds a Qwen3-8B-shaped model (optionally with fewer layers) with seeded N(0, 0.02) bf16 weights drawn on the
 device, prefills a seeded uniform prompt, times the draft and verify forwards with CUDA events, and then runs one
